@@ -1,0 +1,452 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle itself.
+
+Each test names what pins it: an exhaustive comparison with a library routine,
+a closed form, an invariant of the definition (sparse sum over the exact ReLU
+mask = dense sum; all-true mask = dense; partition additivity), a special case
+(full-rank predictor = exact mask), brute force on tiny shapes, or a stored
+hand-derived fixture under tests/golden/.  A plausible mistake in the oracle
+(a dropped term, a wrong sign or index, a transposed operand, the wrong nibble
+order) fails at least one of them.
+"""
+import itertools
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from activation_sparse_decode_gemv_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _layer(lt: inputs.LayerTensors) -> oracle.Layer:
+    return oracle.Layer(**lt.host_arrays())
+
+
+def _manual_layer(W1, W2T, b, P1=None, P2=None, wtype="f32", act="relu", Wg=None, pbias=None):
+    f, d = W1.shape
+    if P1 is None:
+        P1 = np.eye(d, dtype=np.float32)
+        P2 = W1.astype(np.float32)
+    dt = np.float32 if wtype == "f32" else np.float16
+    return oracle.Layer(d=d, f=f, r=P1.shape[0], act=act, wtype=wtype, w_up=W1.astype(dt), w_down_t=W2T.astype(dt),
+                        w_gate=None if Wg is None else Wg.astype(dt), p1=P1.astype(dt), p2=P2.astype(dt),
+                        p_bias=(b if pbias is None else pbias).astype(np.float32),
+                        b_up=None if act == "swiglu" else b.astype(np.float32))
+
+
+# ---------------------------------------------------------------- fp16 codec
+
+def test_half_decode_exhaustive_vs_numpy():
+    """Pin: all 65536 binary16 patterns decode as numpy's float16 -> float64."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = bits.view(np.float16).astype(np.float64)
+    got = np.array([oracle.half_to_double(int(b)) for b in bits])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+    assert np.array_equal(np.signbit(got[~nan]), np.signbit(ref[~nan]))
+
+
+def test_float_to_half_rne_vs_numpy():
+    """Pin: binary32 -> binary16 round-to-nearest-even agrees with numpy's cast,
+    including exact midpoints, subnormals and overflow."""
+    rng = np.random.default_rng(1)
+    vals = [np.float32(v) for v in (0.0, -0.0, 1.0, 65504.0, 65519.99, 65520.0, 70000.0, 2.0 ** -24, 2.0 ** -25,
+                                     3 * 2.0 ** -26, 2.0 ** -14, 1.0 + 2.0 ** -11, 1.0 + 3 * 2.0 ** -11,
+                                     -(1.0 + 2.0 ** -11), 0.1, 1e-8, np.inf, -np.inf)]
+    # exact midpoints between neighbouring fp16 values, both parities
+    h = np.arange(0, 0x7bff, 97, dtype=np.uint16).view(np.float16).astype(np.float64)
+    h2 = (np.arange(0, 0x7bff, 97, dtype=np.uint16) + 1).view(np.float16).astype(np.float64)
+    vals += [np.float32((a + c) / 2) for a, c in zip(h, h2)]
+    vals += list((rng.standard_normal(4000) * np.exp(rng.uniform(-20, 12, 4000))).astype(np.float32))
+    for v in vals:
+        ref = int(np.array([v], np.float32).astype(np.float16).view(np.uint16)[0])
+        assert oracle.float_to_half(v) == ref, (v, hex(ref))
+
+
+def test_golden_half_values():
+    """Pin: hand-derived binary16 values (golden fixture)."""
+    with open(os.path.join(GOLDEN, "half_values.json")) as fh:
+        g = json.load(fh)
+    for bits, val in g["cases"]:
+        assert oracle.half_to_double(int(bits, 16)) == val
+
+
+# ---------------------------------------------------------------- int4
+
+def test_int4_golden_nibble_order():
+    """Pin: golden fixture of packed bytes -> values (element 2k = low nibble)."""
+    with open(os.path.join(GOLDEN, "int4_group.json")) as fh:
+        g = json.load(fh)
+    w = np.array([g["packed"]], np.uint8)
+    sc = np.array([[np.float16(s) for s in g["scales"]]])
+    got = oracle.dequant_row(w, sc, "int4g32", len(g["values"]), 0)
+    assert np.array_equal(got, np.array(g["values"], np.float64))
+
+
+def test_int4_roundtrip_against_quantiser():
+    """Pin: the oracle's dequant of the generator's packing reproduces the
+    generator's own closed-form dequant scale*(q-8) exactly."""
+    w = torch.randn(6, 128, generator=torch.Generator().manual_seed(3)) * 0.02
+    w[2, 32:64] = 0.0  # an all-zero group (scale 0)
+    packed, scales, deq = inputs.quantize_int4g32(w)
+    for row in range(6):
+        got = oracle.dequant_row(packed.numpy(), scales.numpy(), "int4g32", 128, row)
+        assert np.array_equal(got, deq[row].double().numpy())
+    # quantisation error is within half a step of each group's scale
+    err = (deq - w).abs().reshape(6, 4, 32).amax(2)
+    assert torch.all(err <= scales.float() * 0.5 + 1e-7)
+
+
+# ---------------------------------------------------------------- predictor
+
+def test_predict_identity_factor_equals_exact_mask():
+    """Special case: P1 = I (r = d), P2 = W1, bias = b1 gives s = W1 u + b1, the
+    ReLU pre-activation itself (same sum order), so the predicted set is the
+    exact ReLU mask {pre > 0}."""
+    rng = np.random.default_rng(0)
+    f, d = 64, 32
+    W1 = rng.standard_normal((f, d)).astype(np.float32) * 0.2
+    W2T = rng.standard_normal((f, d)).astype(np.float32)
+    b = rng.standard_normal(f).astype(np.float32) * 0.3
+    L = _manual_layer(W1, W2T, b)
+    u = rng.standard_normal((3, d)).astype(np.float32)
+    pr = oracle.predict(L, u)
+    pre = oracle.relu_preact(L, u)
+    assert np.array_equal(pr["s"], pre)
+    for bidx in range(3):
+        assert np.array_equal(pr["idx"][bidx], np.nonzero(pre[bidx] > 0)[0])
+
+
+@pytest.mark.parametrize("kind", ["permutation", "orthogonal"])
+def test_predict_full_rank_factorisation(kind):
+    """Special case: a full-rank factorisation P2 P1 = W1 (P1 = V^T with V a
+    permutation or a random orthogonal matrix, P2 = W1 V) predicts s = W1 u + b1
+    up to rounding.  Catches a transposed P1 or P2 (V V != I in general)."""
+    rng = np.random.default_rng(1)
+    f, d = 48, 24
+    W1 = rng.standard_normal((f, d)) * 0.2
+    b = (rng.standard_normal(f) * 0.3).astype(np.float32)
+    if kind == "permutation":
+        V = np.eye(d)[rng.permutation(d)]
+    else:
+        V, _ = np.linalg.qr(rng.standard_normal((d, d)))
+    P1 = V.T.astype(np.float32)
+    P2 = (W1 @ V).astype(np.float32)
+    L = _manual_layer(W1.astype(np.float32), np.zeros((f, d), np.float32), b, P1=P1, P2=P2)
+    u = rng.standard_normal((2, d)).astype(np.float32)
+    pr = oracle.predict(L, u)
+    exact = (P2.astype(np.float64) @ P1.astype(np.float64)) @ u.astype(np.float64).T + b[:, None]
+    assert np.allclose(pr["s"], exact.T, rtol=0, atol=1e-10)
+    pre = oracle.relu_preact(L, u)
+    tol = 1e-5 if kind == "orthogonal" else 1e-12  # fp32 storage of V for the orthogonal case
+    assert np.max(np.abs(pr["s"] - pre)) < tol
+    for bidx in range(2):
+        sure = np.abs(pre[bidx]) > tol
+        pred = np.zeros(f, bool)
+        pred[pr["idx"][bidx]] = True
+        assert np.array_equal(pred[sure], (pre[bidx] > 0)[sure])
+
+
+def test_predict_closed_form_selectors():
+    """Closed form: P1 row j selects u_{k_j} with weight 2, P2 row i selects h_{j_i}
+    with weight -0.5, so s_i = -u_{k_{j_i}} + b_i exactly.  Checks sign, index
+    and bias handling; s == 0 exactly must not fire (fires iff s > 0)."""
+    d, r, f = 16, 4, 10
+    P1 = np.zeros((r, d), np.float32)
+    ks = [3, 0, 15, 7]
+    for j, k in enumerate(ks):
+        P1[j, k] = 2.0
+    P2 = np.zeros((f, r), np.float32)
+    js = [0, 1, 2, 3, 0, 1, 2, 3, 0, 1]
+    for i, j in enumerate(js):
+        P2[i, j] = -0.5
+    b = np.array([0.5, -1, 0, 2, 1, 0.25, -3, 0, -0.5, 4], np.float32)
+    u = np.arange(d, dtype=np.float32)[None, :] - 5.0  # u_k = k - 5
+    L = _manual_layer(np.zeros((f, d), np.float32), np.zeros((f, d), np.float32), b, P1=P1, P2=P2)
+    pr = oracle.predict(L, u)
+    expect = np.array([-(ks[j] - 5.0) for j in js]) + b
+    assert np.array_equal(pr["s"][0], expect)
+    assert np.array_equal(pr["idx"][0], np.nonzero(expect > 0)[0])
+    assert pr["count"][0] == int((expect > 0).sum())
+    assert 0.0 in expect  # the tie case is exercised
+    assert np.array_equal(pr["h"][0], np.array([2.0 * (k - 5.0) for k in ks]))
+
+
+def test_band_covers_fp32_evaluations():
+    """Pin of the rounding band: single-precision evaluations of s in several
+    summation orders (numpy float32: pairwise, sequential, reversed) stay within
+    the band of the double result for every neuron."""
+    cfg = inputs.CONFIGS["opt7b_f16"].scaled(d=512, f=1024, r=128)
+    lt = inputs.make_layer(cfg, 0, seed=5)
+    L = _layer(lt)
+    x = inputs.make_tokens(cfg, 0, 2, seed=5)
+    u = x.half().numpy()
+    pr = oracle.predict(L, u)
+    P1 = lt.p1.float().numpy()
+    P2 = lt.p2.float().numpy()
+    b = lt.p_bias.numpy()
+    uf = u.astype(np.float32)
+    for bi in range(2):
+        h_pair = P1 @ uf[bi]
+        h_seq = np.zeros(P1.shape[0], np.float32)
+        for k in range(P1.shape[1]):
+            h_seq = (h_seq + P1[:, k] * uf[bi, k]).astype(np.float32)
+        for h in (h_pair, h_seq):
+            s_pair = (P2 @ h.astype(np.float32)).astype(np.float32) + b
+            s_rev = np.zeros(P2.shape[0], np.float32)
+            for j in reversed(range(P2.shape[1])):
+                s_rev = (s_rev + P2[:, j] * h[j]).astype(np.float32)
+            s_rev = (s_rev + b).astype(np.float32)
+            for s32 in (s_pair, s_rev):
+                err = np.abs(s32.astype(np.float64) - pr["s"][bi])
+                assert np.all(err <= pr["band"][bi]), float(np.max(err / pr["band"][bi]))
+    # the band is narrow: well under 1% of neurons are ambiguous
+    assert np.mean(np.abs(pr["s"]) <= pr["band"]) < 0.01
+
+
+# ---------------------------------------------------------------- masked FFN
+
+def _rand_relu_layer(seed=0, f=40, d=24, wtype="f32"):
+    cfg = inputs.CONFIGS["opt_tiny_f32"].scaled(d=d, f=f, r=8, wtype=wtype)
+    return inputs.make_layer(cfg, 0, seed)
+
+
+def test_sparse_all_true_equals_dense_bitwise():
+    """Invariant (definition): the all-true mask gives exactly the dense sum."""
+    for act, wtype in (("relu", "f32"), ("relu", "f16"), ("swiglu", "f16"), ("swiglu", "int4g32")):
+        cfg = inputs.CONFIGS["opt_tiny_f32"].scaled(d=64, f=48, r=8, act=act, wtype=wtype, sort_neurons=True)
+        lt = inputs.make_layer(cfg, 0, 2)
+        L = _layer(lt)
+        u = inputs.layer_input(cfg, inputs.make_tokens(cfg, 0, 3, 2)).numpy()
+        y_all = oracle.ffn_masked(L, u, [np.arange(cfg.f)] * 3)
+        assert np.array_equal(y_all, oracle.ffn_dense(L, u))
+
+
+def test_relu_exact_mask_equals_dense_bitwise():
+    """Invariant: for ReLU the neurons with pre-activation <= 0 contribute
+    exactly +0, so the sparse sum over {pre > 0} equals the dense sum bitwise."""
+    for wtype in ("f32", "f16"):
+        lt = _rand_relu_layer(seed=4, f=96, d=32, wtype=wtype)
+        L = _layer(lt)
+        u = inputs.layer_input(lt.cfg, inputs.make_tokens(lt.cfg, 1, 4, 4)).numpy()
+        pre = oracle.relu_preact(L, u)
+        S = [np.nonzero(pre[b] > 0)[0] for b in range(4)]
+        assert 0 < sum(len(s) for s in S) < 4 * 96
+        assert np.array_equal(oracle.ffn_masked(L, u, S), oracle.ffn_dense(L, u))
+
+
+def test_partition_additivity():
+    """Invariant: sparse(S) + sparse(complement of S) = dense (any activation)."""
+    rng = np.random.default_rng(7)
+    for act in ("relu", "swiglu"):
+        cfg = inputs.CONFIGS["opt_tiny_f32"].scaled(d=32, f=64, r=8, act=act, wtype="f16")
+        lt = inputs.make_layer(cfg, 0, 9)
+        L = _layer(lt)
+        u = inputs.layer_input(cfg, inputs.make_tokens(cfg, 0, 2, 9)).numpy()
+        S = [np.sort(rng.choice(64, 20, replace=False)) for _ in range(2)]
+        Sc = [np.setdiff1d(np.arange(64), s) for s in S]
+        tot = oracle.ffn_masked(L, u, S) + oracle.ffn_masked(L, u, Sc)
+        dense = oracle.ffn_dense(L, u)
+        assert np.allclose(tot, dense, rtol=1e-12, atol=1e-15)
+
+
+def test_empty_set_is_zero():
+    lt = _rand_relu_layer(seed=1)
+    L = _layer(lt)
+    u = inputs.make_tokens(lt.cfg, 0, 2, 1).numpy()
+    y = oracle.ffn_masked(L, u, [np.array([], np.int32)] * 2)
+    assert np.array_equal(y, np.zeros_like(y)) and not np.any(np.signbit(y))
+
+
+def test_single_neuron_closed_form_relu():
+    """Closed form (golden fixture): one-hot W1 rows give pre = u_k + b_i, and
+    y = relu(pre) * W2T_i for a single-neuron set."""
+    with open(os.path.join(GOLDEN, "relu_onehot.json")) as fh:
+        g = json.load(fh)
+    W1 = np.array(g["W1"], np.float32)
+    W2T = np.array(g["W2T"], np.float32)
+    b = np.array(g["b1"], np.float32)
+    u = np.array([g["u"]], np.float32)
+    L = _manual_layer(W1, W2T, b)
+    for case in g["cases"]:
+        y = oracle.ffn_masked(L, u, [np.array(case["set"], np.int32)])
+        assert np.array_equal(y[0], np.array(case["y"], np.float64)), case
+
+
+def test_swiglu_closed_forms():
+    """SiLU pins: with one-hot gate row e_k and up row e_m, phi = SiLU(u_k) u_m.
+    Identities: SiLU(z) - SiLU(-z) = z; SiLU(0) = 0; SiLU(z) -> z for large z
+    and -> 0 for very negative z.  (exp itself comes from libm: parity of the
+    SiLU value beyond these identities is unpinned.)"""
+    d, f = 8, 1
+    Wg = np.zeros((f, d), np.float32); Wg[0, 2] = 1.0
+    Wu = np.zeros((f, d), np.float32); Wu[0, 5] = 1.0
+    W2T = np.zeros((f, d), np.float32); W2T[0, 0] = 1.0
+    L = _manual_layer(Wu, W2T, np.zeros(f, np.float32), act="swiglu", Wg=Wg, wtype="f16")
+    for z in (0.5, 1.0, 2.75, 6.0, 0.125):
+        u = np.zeros((2, d), np.float32)
+        u[0, 2], u[1, 2] = z, -z
+        u[:, 5] = 1.0
+        phi = oracle.neuron_phi(L, u.astype(np.float16))
+        assert abs((phi[0, 0] - phi[1, 0]) - z) < 1e-15
+        assert 0 < phi[0, 0] < z and -0.3 < phi[1, 0] < 0
+    u = np.zeros((3, d), np.float16)
+    u[0, 5] = 1.0
+    u[1, 2], u[1, 5] = 20.0, 1.0
+    u[2, 2], u[2, 5] = -60.0, 1.0
+    phi = oracle.neuron_phi(L, u)
+    assert phi[0, 0] == 0.0
+    assert abs(phi[1, 0] - 20.0) < 1e-6
+    assert abs(phi[2, 0]) < 1e-20
+
+
+def test_dense_matches_library_matmul():
+    """Library reduction: the dense ReLU / SwiGLU FFN equals the same formula
+    written with numpy matmuls (a different summation routine)."""
+    for act in ("relu", "swiglu"):
+        cfg = inputs.CONFIGS["opt_tiny_f32"].scaled(d=64, f=96, r=8, act=act, wtype="f16")
+        lt = inputs.make_layer(cfg, 0, 11)
+        L = _layer(lt)
+        u = inputs.layer_input(cfg, inputs.make_tokens(cfg, 0, 2, 11)).numpy()
+        U = u.astype(np.float64)
+        W2T = lt.w_down_t.double().numpy()
+        if act == "relu":
+            phi = np.maximum(U @ lt.w_up.double().numpy().T + lt.b_up.double().numpy(), 0)
+        else:
+            g = U @ lt.w_gate.double().numpy().T
+            phi = g / (1 + np.exp(-g)) * (U @ lt.w_up.double().numpy().T)
+        assert np.allclose(oracle.ffn_dense(L, u), phi @ W2T, rtol=1e-12, atol=1e-14)
+
+
+def test_brute_force_all_masks_tiny():
+    """Brute force: f = 10 neurons, every one of the 2^10 masks equals the sum
+    of that mask's per-neuron terms phi_i W2T_i (terms from single-neuron sets,
+    checked against an explicit per-neuron computation)."""
+    for act in ("relu", "swiglu"):
+        cfg = inputs.CONFIGS["opt_tiny_f32"].scaled(d=8, f=10, r=4, act=act, wtype="f32")
+        lt = inputs.make_layer(cfg, 0, 13)
+        L = _layer(lt)
+        u = inputs.make_tokens(cfg, 0, 1, 13).numpy()
+        terms = np.stack([oracle.ffn_masked(L, u, [np.array([i], np.int32)])[0] for i in range(10)])
+        # per-neuron terms by explicit loops (independent of the C code path)
+        W1 = lt.w_up.double().numpy(); W2T = lt.w_down_t.double().numpy(); uu = u[0].astype(np.float64)
+        for i in range(10):
+            if act == "relu":
+                pre = sum(W1[i, k] * uu[k] for k in range(8)) + float(lt.b_up[i])
+                phi = max(pre, 0.0)
+            else:
+                Wg = lt.w_gate.double().numpy()
+                g = sum(Wg[i, k] * uu[k] for k in range(8))
+                v = sum(W1[i, k] * uu[k] for k in range(8))
+                phi = g / (1 + np.exp(-g)) * v
+            assert np.allclose(terms[i], phi * W2T[i], rtol=1e-13, atol=1e-16)
+        for m in range(1 << 10):
+            S = np.array([i for i in range(10) if m >> i & 1], np.int32)
+            y = oracle.ffn_masked(L, u, [S])[0]
+            assert np.allclose(y, terms[S].sum(0) if len(S) else 0.0, rtol=1e-12, atol=1e-15)
+
+
+def test_neuron_permutation_invariance():
+    """Invariant: permuting the neuron storage order (rows of W1, W2T, b1) and
+    mapping the index set accordingly leaves y unchanged up to rounding."""
+    lt = _rand_relu_layer(seed=21, f=64, d=32)
+    L = _layer(lt)
+    u = inputs.make_tokens(lt.cfg, 0, 2, 21).numpy()
+    perm = np.random.default_rng(0).permutation(64)
+    inv = np.argsort(perm)
+    a = lt.host_arrays()
+    Lp = oracle.Layer(**{**a, "w_up": a["w_up"][perm], "w_down_t": a["w_down_t"][perm],
+                         "b_up": a["b_up"][perm], "p2": a["p2"][perm], "p_bias": a["p_bias"][perm]})
+    S = [np.array([1, 5, 6, 30, 63], np.int32), np.arange(0, 64, 3, dtype=np.int32)]
+    Sp = [np.sort(inv[s]).astype(np.int32) for s in S]
+    assert np.allclose(oracle.ffn_masked(L, u, S), oracle.ffn_masked(Lp, u, Sp), rtol=1e-13, atol=1e-16)
+    # the predicted sets map onto each other too
+    pa, pb = oracle.predict(L, u), oracle.predict(Lp, u)
+    for b in range(2):
+        assert np.array_equal(np.sort(perm[pb["idx"][b]]), pa["idx"][b])
+
+
+def test_masked_rejects_bad_index_lists():
+    lt = _rand_relu_layer(seed=2)
+    L = _layer(lt)
+    u = inputs.make_tokens(lt.cfg, 0, 1, 2).numpy()
+    for bad in ([3, 3], [5, 2], [0, 40], [-1]):
+        with pytest.raises(oracle.OracleError):
+            oracle.ffn_masked(L, u, [np.array(bad, np.int32)])
+
+
+# ---------------------------------------------------------------- RMS norm and stack
+
+def test_rmsnorm_golden():
+    """Closed forms (golden fixture): constant and alternating vectors, zeros."""
+    with open(os.path.join(GOLDEN, "rmsnorm.json")) as fh:
+        g = json.load(fh)
+    for case in g["cases"]:
+        u, _ = oracle.rmsnorm_f16(np.array([case["x"]], np.float32))
+        assert np.array_equal(u[0].astype(np.float64), np.array(case["u"], np.float64)), case
+
+
+def test_rmsnorm_unit_rms_and_scale_invariance():
+    """The normalised vector has RMS 1 up to fp16 rounding, and scaling x by a
+    power of two changes u by at most one fp16 ulp (only through the epsilon,
+    which moves the denominator by about an ulp), and only rarely."""
+    x = np.random.default_rng(3).standard_normal((3, 512)).astype(np.float32) * 5
+    u, m = oracle.rmsnorm_f16(x)
+    rms = np.sqrt(np.mean(u.astype(np.float64) ** 2, axis=1))
+    assert np.all(np.abs(rms - 1) < 2e-3)
+    u4, _ = oracle.rmsnorm_f16(x * 4)
+    diff = np.abs(u.view(np.uint16).astype(np.int32) - u4.view(np.uint16).astype(np.int32))
+    assert diff.max() <= 1 and np.mean(diff) < 0.02
+    assert np.all(m >= 0) and np.all(m < 0.5)
+
+
+def test_stack_single_layer_composition():
+    """A one-layer stack is rmsnorm -> predict -> masked FFN -> x + y."""
+    cfg = inputs.CONFIGS["opt30b_stack_f16"].scaled(d=64, f=256, r=16, n_layers=1)
+    lt = inputs.make_layer(cfg, 0, 3)
+    L = _layer(lt)
+    x = inputs.make_tokens(cfg, 0, 2, 3).numpy()
+    st = oracle.stack([L], x)
+    u, _ = oracle.rmsnorm_f16(x)
+    pr = oracle.predict(L, u)
+    y = oracle.ffn_masked(L, u, pr["idx"])
+    assert np.array_equal(st["y"][0], y)
+    assert np.array_equal(st["x"], (x.astype(np.float64) + y).astype(np.float32))
+    for b in range(2):
+        assert np.array_equal(st["idx"][0][b], pr["idx"][b])
+
+
+def test_stack_zero_down_projection_keeps_x():
+    cfg = inputs.CONFIGS["opt30b_stack_f16"].scaled(d=64, f=128, r=16, n_layers=2)
+    Ls = []
+    for l in range(2):
+        a = inputs.make_layer(cfg, l, 4).host_arrays()
+        a["w_down_t"] = np.zeros_like(a["w_down_t"])
+        Ls.append(oracle.Layer(**a))
+    x = inputs.make_tokens(cfg, 0, 1, 4).numpy()
+    st = oracle.stack(Ls, x)
+    assert np.array_equal(st["x"], x)
+
+
+# ---------------------------------------------------------------- generator checks
+
+@pytest.mark.parametrize("name,mean_p", [("opt7b_f16", 0.10), ("opt30b_stack_f16", 0.03),
+                                         ("llama13b_swiglu_f16", 0.43), ("llama70b_swiglu_int4", 0.50)])
+def test_generator_firing_rate(name, mean_p):
+    """Generator check (not the method): over seeded N(0, I) tokens the mean
+    predicted-active fraction is within 15% of the configured target."""
+    cfg = inputs.CONFIGS[name].scaled(d=256, f=2048, r=64)
+    lt = inputs.make_layer(cfg, 0, 17)
+    L = _layer(lt)
+    x = inputs.make_tokens(cfg, 0, 64, 17)
+    pr = oracle.predict(L, x.half().numpy())
+    frac = pr["count"].mean() / cfg.f
+    assert abs(frac - mean_p) <= 0.15 * mean_p, frac
+    # hot prefix really is hotter than the tail
+    hot = np.mean([np.mean(i < lt.hot_prefix) for i in pr["idx"]])
+    assert hot > 0.2
