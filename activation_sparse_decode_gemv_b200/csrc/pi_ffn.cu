@@ -1,0 +1,471 @@
+// pi_ffn.cu -- C ABI of the predictor-gated sparse FFN decode library: host
+// validation, workspace layout and kernel dispatch.  The declarations and
+// argument contracts live in include/pi_ffn.h.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <new>
+
+#include "pi_ffn.h"
+#include "pi_kernels.cuh"
+
+struct pi_ffn {
+  pi_ffn_desc d;
+  int H;       // hot prefix rounded down to a multiple of 32
+  int nwords;  // ceil(f / 32)
+};
+
+namespace {
+
+constexpr int kMaxBatch = 32;
+constexpr int kMaxD = 16384;
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Workspace layout for a call at batch B on layers with the given maxima.
+// [0, 256): status region (int status, int union count, ...).
+struct WsLayout {
+  size_t h, u, mask, uwords, uprefix, ulist, partial, total;
+  int G;
+};
+
+int device_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+WsLayout ws_layout(int dmax, int fmax, int rmax, int B, int G) {
+  WsLayout L{};
+  size_t o = 256;
+  const size_t nw = (size_t)(fmax + 31) / 32;
+  L.h = o;
+  o = align_up(o + (size_t)B * rmax * 4, 256);
+  L.u = o;
+  o = align_up(o + (size_t)B * dmax * 2, 256);
+  L.mask = o;
+  o = align_up(o + (size_t)B * nw * 4, 256);
+  L.uwords = o;
+  o = align_up(o + nw * 4, 256);
+  L.uprefix = o;
+  o = align_up(o + (nw + 1) * 4, 256);
+  L.ulist = o;
+  o = align_up(o + (size_t)fmax * 4, 256);
+  L.partial = o;
+  o = align_up(o + (size_t)G * B * dmax * 4, 256);
+  L.total = o;
+  L.G = G;
+  return L;
+}
+
+struct Ws {
+  WsLayout L;
+  char *base;
+  int *status() const { return reinterpret_cast<int *>(base); }
+  int32_t *ucount() const { return reinterpret_cast<int32_t *>(base) + 1; }
+  float *h() const { return reinterpret_cast<float *>(base + L.h); }
+  __half *u() const { return reinterpret_cast<__half *>(base + L.u); }
+  uint32_t *mask() const { return reinterpret_cast<uint32_t *>(base + L.mask); }
+  uint32_t *uwords() const { return reinterpret_cast<uint32_t *>(base + L.uwords); }
+  int32_t *uprefix() const { return reinterpret_cast<int32_t *>(base + L.uprefix); }
+  int32_t *ulist() const { return reinterpret_cast<int32_t *>(base + L.ulist); }
+  float *partial() const { return reinterpret_cast<float *>(base + L.partial); }
+};
+
+pi_status get_ws(const pi_ffn *const *layers, int n, int B, void *ws, size_t ws_bytes, Ws *out) {
+  if (!ws) return PI_ERR_WORKSPACE;
+  if (!aligned16(ws)) return PI_ERR_MISALIGNED;
+  int dmax = 0, fmax = 0, rmax = 0;
+  for (int i = 0; i < n; ++i) {
+    dmax = dmax > layers[i]->d.d_model ? dmax : layers[i]->d.d_model;
+    fmax = fmax > layers[i]->d.d_ffn ? fmax : layers[i]->d.d_ffn;
+    rmax = rmax > layers[i]->d.rank ? rmax : layers[i]->d.rank;
+  }
+  const int G = device_sm_count();
+  if (G <= 0) return PI_ERR_CUDA;
+  out->L = ws_layout(dmax, fmax, rmax, B, G);
+  out->base = static_cast<char *>(ws);
+  return out->L.total <= ws_bytes ? PI_OK : PI_ERR_WORKSPACE;
+}
+
+// ---------------------------------------------------------------- launching
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+inline int nb_for(int B) { return B <= 1 ? 1 : B <= 2 ? 2 : B <= 4 ? 4 : 8; }
+inline int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+template <int NB>
+cudaError_t pred_h_nb(int pt, dim3 g, cudaStream_t st, const void *p1, const void *u, int d, int r, int B, float *h) {
+  return pt == PI_W_F32 ? launch(pi::pred_h_kernel<NB, pi::W_F32>, g, dim3(256), st, p1, u, d, r, B, h)
+                        : launch(pi::pred_h_kernel<NB, pi::W_F16>, g, dim3(256), st, p1, u, d, r, B, h);
+}
+template <int NB>
+cudaError_t pred_s_nb(int pt, dim3 g, cudaStream_t st, const void *p2, const float *h, const float *bias, int f, int r,
+                      int B, uint32_t *mask, int nw) {
+  return pt == PI_W_F32 ? launch(pi::pred_s_kernel<NB, pi::W_F32>, g, dim3(256), st, p2, h, bias, f, r, B, mask, nw)
+                        : launch(pi::pred_s_kernel<NB, pi::W_F16>, g, dim3(256), st, p2, h, bias, f, r, B, mask, nw);
+}
+
+// gather kernel dispatch: NB tokens per CTA row, GPT column groups per thread
+template <int NB, int WT, int ACT>
+cudaError_t gather_gpt(int gpt, dim3 g, dim3 b, cudaStream_t st, const pi::FfnArgs &a) {
+  switch (gpt) {
+  case 1:
+    return launch(pi::ffn_gather_kernel<NB, WT, ACT, 1>, g, b, st, a);
+  case 2:
+    if constexpr (NB * 2 <= 8) return launch(pi::ffn_gather_kernel<NB, WT, ACT, 2>, g, b, st, a);
+    break;
+  case 4:
+    if constexpr (NB * 4 <= 8) return launch(pi::ffn_gather_kernel<NB, WT, ACT, 4>, g, b, st, a);
+    break;
+  }
+  return cudaErrorInvalidConfiguration;
+}
+template <int NB, int WT>
+cudaError_t gather_act(int act, int gpt, dim3 g, dim3 b, cudaStream_t st, const pi::FfnArgs &a) {
+  return act == PI_ACT_RELU ? gather_gpt<NB, WT, pi::ACT_RELU>(gpt, g, b, st, a)
+                            : gather_gpt<NB, WT, pi::ACT_SWIGLU>(gpt, g, b, st, a);
+}
+template <int NB>
+cudaError_t gather_wt(int wt, int act, int gpt, dim3 g, dim3 b, cudaStream_t st, const pi::FfnArgs &a) {
+  switch (wt) {
+  case PI_W_F32:
+    return gather_act<NB, pi::W_F32>(act, gpt, g, b, st, a);
+  case PI_W_F16:
+    return gather_act<NB, pi::W_F16>(act, gpt, g, b, st, a);
+  default:
+    return gather_act<NB, pi::W_INT4>(act, gpt, g, b, st, a);
+  }
+}
+
+// Token group size and column groups per thread for the gather kernel:
+// NB * GPT <= 8 (at most 64 fp32 accumulators per thread) and the CTA covers
+// the d/8 column groups with at most 512 threads (128 registers each).
+void gather_shape(int B, int d, int *nb, int *gpt, int *threads) {
+  const int ngroups = d / 8;
+  for (int n = nb_for(B); n >= 1; n >>= 1) {
+    for (int g = 1; g <= 4 && n * g <= 8; g <<= 1) {
+      const int maxt = 512;
+      int t = (cdiv(ngroups, g) + 31) / 32 * 32;
+      if (t < 128) t = 128;
+      if (t <= maxt) {
+        *nb = n;
+        *gpt = g;
+        *threads = t;
+        return;
+      }
+    }
+  }
+  *nb = 1;
+  *gpt = 4;
+  *threads = 512;
+}
+
+bool want_dense(const pi_ffn *h, int B, unsigned flags) {
+  if (h->H <= 0) return false;
+  if (flags & PI_FFN_HOT_DENSE) return true;
+  if (flags & PI_FFN_HOT_INDEX) return false;
+  const double p = h->d.hot_p_mean;
+  if (!(p > 0.0)) return false;
+  return 1.0 - std::pow(1.0 - (p < 1.0 ? p : 1.0), (double)B) >= 0.75;
+}
+
+#define PI_CUDA(call)                      \
+  do {                                     \
+    if ((call) != cudaSuccess) return PI_ERR_CUDA; \
+  } while (0)
+
+// steps 1-2: predictor, mask words, compaction (idx/count optional)
+pi_status run_predict(const pi_ffn *h, const void *u, int B, int32_t *idx, int idx_stride, int32_t *count, const Ws &w,
+                      cudaStream_t st) {
+  const pi_ffn_desc &D = h->d;
+  const int nb = nb_for(B);
+  const dim3 gh(cdiv(D.rank, 8), cdiv(B, nb)), gs(h->nwords, cdiv(B, nb));
+  cudaError_t e;
+  switch (nb) {
+  case 1:
+    e = pred_h_nb<1>(D.ptype, gh, st, D.p1, u, D.d_model, D.rank, B, w.h());
+    break;
+  case 2:
+    e = pred_h_nb<2>(D.ptype, gh, st, D.p1, u, D.d_model, D.rank, B, w.h());
+    break;
+  case 4:
+    e = pred_h_nb<4>(D.ptype, gh, st, D.p1, u, D.d_model, D.rank, B, w.h());
+    break;
+  default:
+    e = pred_h_nb<8>(D.ptype, gh, st, D.p1, u, D.d_model, D.rank, B, w.h());
+  }
+  PI_CUDA(e);
+  switch (nb) {
+  case 1:
+    e = pred_s_nb<1>(D.ptype, gs, st, D.p2, w.h(), D.p_bias, D.d_ffn, D.rank, B, w.mask(), h->nwords);
+    break;
+  case 2:
+    e = pred_s_nb<2>(D.ptype, gs, st, D.p2, w.h(), D.p_bias, D.d_ffn, D.rank, B, w.mask(), h->nwords);
+    break;
+  case 4:
+    e = pred_s_nb<4>(D.ptype, gs, st, D.p2, w.h(), D.p_bias, D.d_ffn, D.rank, B, w.mask(), h->nwords);
+    break;
+  default:
+    e = pred_s_nb<8>(D.ptype, gs, st, D.p2, w.h(), D.p_bias, D.d_ffn, D.rank, B, w.mask(), h->nwords);
+  }
+  PI_CUDA(e);
+  PI_CUDA(launch(pi::compact_kernel, dim3(B + 1), dim3(1024), st, (const uint32_t *)w.mask(), h->nwords, idx_stride, B,
+                 idx, count, w.uwords(), w.uprefix(), w.ulist(), w.ucount()));
+  return PI_OK;
+}
+
+// caller id lists -> mask words and union
+pi_status run_sets(const pi_ffn *h, const int32_t *idx, const int32_t *count, int B, const Ws &w, cudaStream_t st) {
+  PI_CUDA(cudaMemsetAsync(w.mask(), 0, (size_t)B * h->nwords * 4, st));
+  const int f = h->d.d_ffn;
+  PI_CUDA(launch(pi::idx_to_mask_kernel, dim3(cdiv(f, 256) < 64 ? cdiv(f, 256) : 64, B), dim3(256), st, idx, count, f,
+                 w.mask(), h->nwords, w.status()));
+  PI_CUDA(launch(pi::compact_kernel, dim3(B + 1), dim3(1024), st, (const uint32_t *)w.mask(), h->nwords, 0, B,
+                 (int32_t *)nullptr, (int32_t *)nullptr, w.uwords(), w.uprefix(), w.ulist(), w.ucount()));
+  return PI_OK;
+}
+
+// steps 3-4 over the union in the workspace; out (=, +=) y
+pi_status run_ffn(const pi_ffn *h, const void *u, int B, float *out, int accumulate, unsigned flags, const Ws &w,
+                  cudaStream_t st) {
+  const pi_ffn_desc &D = h->d;
+  pi::FfnArgs a{};
+  a.w_up = D.w_up;
+  a.w_gate = D.w_gate;
+  a.w_down_t = D.w_down_t;
+  a.s_up = reinterpret_cast<const __half *>(D.s_up);
+  a.s_gate = reinterpret_cast<const __half *>(D.s_gate);
+  a.s_down_t = reinterpret_cast<const __half *>(D.s_down_t);
+  a.b_up = D.b_up;
+  a.u = u;
+  a.d = D.d_model;
+  a.f = D.d_ffn;
+  a.B = B;
+  a.mask = w.mask();
+  a.nwords = h->nwords;
+  a.ulist = w.ulist();
+  a.ucount = w.ucount();
+  a.uprefix = w.uprefix();
+  a.hot_dense = want_dense(h, B, flags) ? 1 : 0;
+  a.H = h->H;
+  a.partial = w.partial();
+  int nb, gpt, threads;
+  gather_shape(B, D.d_model, &nb, &gpt, &threads);
+  const dim3 g(w.L.G, cdiv(B, nb)), blk(threads);
+  cudaError_t e;
+  switch (nb) {
+  case 1:
+    e = gather_wt<1>(D.wtype, D.act, gpt, g, blk, st, a);
+    break;
+  case 2:
+    e = gather_wt<2>(D.wtype, D.act, gpt, g, blk, st, a);
+    break;
+  case 4:
+    e = gather_wt<4>(D.wtype, D.act, gpt, g, blk, st, a);
+    break;
+  default:
+    e = gather_wt<8>(D.wtype, D.act, gpt, g, blk, st, a);
+  }
+  PI_CUDA(e);
+  const int n_elem = B * D.d_model;
+  PI_CUDA(launch(pi::reduce_kernel, dim3(cdiv(n_elem, 256)), dim3(256), st, (const float *)w.partial(), w.L.G,
+                 (const int32_t *)w.ucount(), (const int32_t *)w.uprefix(), a.hot_dense, h->H, n_elem, out, accumulate));
+  return PI_OK;
+}
+
+pi_status check_call(const pi_ffn *h, int B) {
+  if (!h) return PI_ERR_INVALID_ARG;
+  if (B < 0 || B > kMaxBatch) return PI_ERR_UNSUPPORTED;
+  return PI_OK;
+}
+
+}  // namespace
+
+// ====================================================================== API
+
+extern "C" {
+
+pi_status pi_ffn_create(const pi_ffn_desc *desc, pi_ffn_t *out) {
+  if (!desc || !out) return PI_ERR_INVALID_ARG;
+  const pi_ffn_desc &D = *desc;
+  if (D.d_model <= 0 || D.d_ffn <= 0 || D.rank <= 0) return PI_ERR_INVALID_ARG;
+  if (D.act != PI_ACT_RELU && D.act != PI_ACT_SWIGLU) return PI_ERR_INVALID_ARG;
+  if (D.wtype != PI_W_F32 && D.wtype != PI_W_F16 && D.wtype != PI_W_INT4G32) return PI_ERR_INVALID_ARG;
+  if (D.ptype != PI_W_F32 && D.ptype != PI_W_F16) return PI_ERR_INVALID_ARG;
+  if (!D.w_up || !D.w_down_t || !D.p1 || !D.p2 || !D.p_bias) return PI_ERR_INVALID_ARG;
+  if (D.act == PI_ACT_RELU && !D.b_up) return PI_ERR_INVALID_ARG;
+  if (D.act == PI_ACT_SWIGLU && !D.w_gate) return PI_ERR_INVALID_ARG;
+  if (D.wtype == PI_W_INT4G32 && (!D.s_up || !D.s_down_t || (D.act == PI_ACT_SWIGLU && !D.s_gate)))
+    return PI_ERR_INVALID_ARG;
+  if (D.hot_prefix < 0 || D.hot_prefix > D.d_ffn) return PI_ERR_INVALID_ARG;
+  // the FFN input u is fp32 exactly when the weights are fp32; the predictor
+  // factors share u's type
+  if ((D.wtype == PI_W_F32) != (D.ptype == PI_W_F32)) return PI_ERR_UNSUPPORTED;
+  if (D.d_model % 8 || D.d_model > kMaxD) return PI_ERR_UNSUPPORTED;
+  if (D.wtype == PI_W_INT4G32 && D.d_model % 32) return PI_ERR_UNSUPPORTED;
+  if (D.rank % (D.ptype == PI_W_F32 ? 4 : 8)) return PI_ERR_UNSUPPORTED;
+  const void *ptrs[] = {D.w_up, D.w_gate, D.w_down_t, D.s_up, D.s_gate, D.s_down_t, D.b_up, D.p1, D.p2, D.p_bias};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return PI_ERR_MISALIGNED;
+  pi_ffn *h = new (std::nothrow) pi_ffn;
+  if (!h) return PI_ERR_INVALID_ARG;
+  h->d = D;
+  h->H = D.hot_prefix & ~31;
+  h->nwords = (D.d_ffn + 31) / 32;
+  *out = h;
+  return PI_OK;
+}
+
+void pi_ffn_destroy(pi_ffn_t h) { delete h; }
+
+pi_status pi_workspace_size(const pi_ffn_t *layers, int n_layers, int max_batch, size_t *bytes) {
+  if (!layers || n_layers <= 0 || !bytes) return PI_ERR_INVALID_ARG;
+  if (max_batch <= 0 || max_batch > kMaxBatch) return PI_ERR_UNSUPPORTED;
+  for (int i = 0; i < n_layers; ++i)
+    if (!layers[i]) return PI_ERR_INVALID_ARG;
+  int dmax = 0, fmax = 0, rmax = 0;
+  for (int i = 0; i < n_layers; ++i) {
+    dmax = dmax > layers[i]->d.d_model ? dmax : layers[i]->d.d_model;
+    fmax = fmax > layers[i]->d.d_ffn ? fmax : layers[i]->d.d_ffn;
+    rmax = rmax > layers[i]->d.rank ? rmax : layers[i]->d.rank;
+  }
+  const int G = device_sm_count();
+  if (G <= 0) return PI_ERR_CUDA;
+  *bytes = ws_layout(dmax, fmax, rmax, max_batch, G).total;
+  return PI_OK;
+}
+
+pi_status pi_workspace_init(void *ws, size_t ws_bytes, pi_stream_t stream) {
+  if (!ws || ws_bytes == 0) return PI_ERR_INVALID_ARG;
+  if (!aligned16(ws)) return PI_ERR_MISALIGNED;
+  return cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream) == cudaSuccess ? PI_OK : PI_ERR_CUDA;
+}
+
+pi_status pi_predict(pi_ffn_t h, const void *u, int B, int32_t *idx, int32_t *count, void *ws, size_t ws_bytes,
+                     pi_stream_t stream) {
+  pi_status s = check_call(h, B);
+  if (s != PI_OK) return s;
+  if (!u || !idx || !count) return PI_ERR_INVALID_ARG;
+  if (!aligned16(u) || !aligned16(idx) || !aligned16(count)) return PI_ERR_MISALIGNED;
+  if (B == 0) return PI_OK;
+  Ws w;
+  const pi_ffn *L[1] = {h};
+  if ((s = get_ws(L, 1, B, ws, ws_bytes, &w)) != PI_OK) return s;
+  return run_predict(h, u, B, idx, h->d.d_ffn, count, w, (cudaStream_t)stream);
+}
+
+pi_status pi_sparse_ffn(pi_ffn_t h, const void *u, int B, const int32_t *idx, const int32_t *count, float *y,
+                        unsigned flags, void *ws, size_t ws_bytes, pi_stream_t stream) {
+  pi_status s = check_call(h, B);
+  if (s != PI_OK) return s;
+  if (!u || !idx || !count || !y) return PI_ERR_INVALID_ARG;
+  if (!aligned16(u) || !aligned16(idx) || !aligned16(count) || !aligned16(y)) return PI_ERR_MISALIGNED;
+  if (flags & ~7u) return PI_ERR_INVALID_ARG;
+  if (B == 0) return PI_OK;
+  Ws w;
+  const pi_ffn *L[1] = {h};
+  if ((s = get_ws(L, 1, B, ws, ws_bytes, &w)) != PI_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  if ((s = run_sets(h, idx, count, B, w, st)) != PI_OK) return s;
+  return run_ffn(h, u, B, y, (flags & PI_FFN_ACCUMULATE) ? 1 : 0, flags, w, st);
+}
+
+pi_status pi_decode_ffn(pi_ffn_t h, const void *u, int B, float *y, int32_t *idx, int32_t *count, unsigned flags,
+                        void *ws, size_t ws_bytes, pi_stream_t stream) {
+  pi_status s = check_call(h, B);
+  if (s != PI_OK) return s;
+  if (!u || !y) return PI_ERR_INVALID_ARG;
+  if (!aligned16(u) || !aligned16(y) || (idx && !aligned16(idx)) || (count && !aligned16(count)))
+    return PI_ERR_MISALIGNED;
+  if (flags & ~7u) return PI_ERR_INVALID_ARG;
+  if (B == 0) return PI_OK;
+  Ws w;
+  const pi_ffn *L[1] = {h};
+  if ((s = get_ws(L, 1, B, ws, ws_bytes, &w)) != PI_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  if ((s = run_predict(h, u, B, idx, h->d.d_ffn, count, w, st)) != PI_OK) return s;
+  return run_ffn(h, u, B, y, (flags & PI_FFN_ACCUMULATE) ? 1 : 0, flags, w, st);
+}
+
+pi_status pi_decode_ffn_stack(const pi_ffn_t *layers, int L, float *x, int B, int32_t *idx_trace,
+                              int32_t *count_trace, unsigned flags, void *ws, size_t ws_bytes, pi_stream_t stream) {
+  if (!layers || L <= 0 || !x) return PI_ERR_INVALID_ARG;
+  if (B < 0 || B > kMaxBatch) return PI_ERR_UNSUPPORTED;
+  if (!aligned16(x) || (idx_trace && !aligned16(idx_trace)) || (count_trace && !aligned16(count_trace)))
+    return PI_ERR_MISALIGNED;
+  if (flags & ~6u) return PI_ERR_INVALID_ARG;
+  int fmax = 0;
+  for (int l = 0; l < L; ++l) {
+    if (!layers[l]) return PI_ERR_INVALID_ARG;
+    if (layers[l]->d.d_model != layers[0]->d.d_model) return PI_ERR_UNSUPPORTED;
+    if (layers[l]->d.wtype == PI_W_F32) return PI_ERR_UNSUPPORTED;
+    fmax = fmax > layers[l]->d.d_ffn ? fmax : layers[l]->d.d_ffn;
+  }
+  if (B == 0) return PI_OK;
+  Ws w;
+  pi_status s = get_ws(layers, L, B, ws, ws_bytes, &w);
+  if (s != PI_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int d = layers[0]->d.d_model;
+  for (int l = 0; l < L; ++l) {
+    PI_CUDA(launch(pi::rmsnorm_kernel, dim3(B), dim3(256), st, (const float *)x, d, w.u()));
+    int32_t *idx = idx_trace ? idx_trace + (size_t)l * B * fmax : nullptr;
+    int32_t *cnt = count_trace ? count_trace + (size_t)l * B : nullptr;
+    if ((s = run_predict(layers[l], w.u(), B, idx, fmax, cnt, w, st)) != PI_OK) return s;
+    if ((s = run_ffn(layers[l], w.u(), B, x, 1, flags, w, st)) != PI_OK) return s;
+  }
+  return PI_OK;
+}
+
+pi_status pi_get_device_status(void *ws, pi_stream_t stream, int *code) {
+  if (!ws || !code) return PI_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return PI_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return PI_ERR_CUDA;
+  if (v != 0 && cudaMemset(ws, 0, sizeof(int)) != cudaSuccess) return PI_ERR_CUDA;
+  *code = v;
+  return PI_OK;
+}
+
+const char *pi_status_string(pi_status s) {
+  switch (s) {
+  case PI_OK:
+    return "ok";
+  case PI_ERR_INVALID_ARG:
+    return "invalid argument";
+  case PI_ERR_UNSUPPORTED:
+    return "unsupported shape or type";
+  case PI_ERR_MISALIGNED:
+    return "pointer not 16-byte aligned";
+  case PI_ERR_CUDA:
+    return "CUDA runtime error";
+  case PI_ERR_TIMEOUT:
+    return "device wait timed out";
+  case PI_ERR_DEVICE_STATUS:
+    return "device-side argument error";
+  case PI_ERR_WORKSPACE:
+    return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,414 @@
+#!/usr/bin/env python
+"""Benchmark of the sparse-FFN decode hot path on B200.
+
+One step = one full pass of the decode path over one token batch of one FFN
+layer: predictor (h = P1 u, s = P2 h + b, threshold), compaction of the active
+ids, gathered up/gate rows with the activation, gathered down-projection rows,
+reduction.  Default workload: the OPT-7B-shaped fp16 ReLU layer (d = 4096,
+f = 16384, rank-1024 predictor, mean firing rate 10%, hot prefix 20%) at
+batch 1.  Steps rotate through 8 independently seeded layer replicas (2.5 GB,
+far above the 126 MB L2) and 32 seeded tokens, so weights come from HBM.
+
+Metric: achieved HBM GB/s over the bytes the step must touch (predictor
+weights + up rows of the predicted union + down rows of the neurons with a
+nonzero activation + token in / y out), with us per layer alongside.  Timed
+with CUDA events around graph replays; N > 1 GPUs run independent replicas
+(weak scaling, no collective on the data path) and the time is the maximum
+over ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np
+import torch
+
+from activation_sparse_decode_gemv_b200 import inputs
+
+KERNELS_PER_STEP = 5  # pred_h, pred_s, compact, gather, reduce
+
+
+def parse(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40000)
+    ap.add_argument("--warmup", type=int, default=4000)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="opt7b_f16")
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--replicas", type=int, default=8)
+    ap.add_argument("--tokens", type=int, default=32)
+    ap.add_argument("--flags", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=2000)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-seconds", type=float, default=90.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--json-out", default=None)
+    return ap.parse_args(argv)
+
+
+# ----------------------------------------------------------------------------- distributed plumbing
+
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(value: float, world: int) -> float:
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    dev = torch.device("cuda") if dist.get_backend() == "nccl" else torch.device("cpu")
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(value: float, world: int) -> float:
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    dev = torch.device("cuda") if dist.get_backend() == "nccl" else torch.device("cpu")
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def aggregate(bytes_per_rank: float, seconds_per_rank: float, world: int):
+    """Whole-job GB/s: all ranks' bytes over the slowest rank's time."""
+    t = max_over_ranks(seconds_per_rank, world)
+    b = sum_over_ranks(bytes_per_rank, world)
+    return b / t / 1e9, t
+
+
+# ----------------------------------------------------------------------------- bytes of a step
+
+def row_bytes(cfg: inputs.Config) -> int:
+    if cfg.wtype == "f32":
+        return cfg.d * 4
+    if cfg.wtype == "f16":
+        return cfg.d * 2
+    return cfg.d // 2 + (cfg.d // 32) * 2
+
+
+def predictor_bytes(cfg: inputs.Config) -> int:
+    e = 4 if cfg.wtype == "f32" else 2
+    return (cfg.r * cfg.d + cfg.f * cfg.r) * e + 4 * cfg.f
+
+
+def step_bytes(cfg: inputs.Config, B: int, n_up_rows: int, n_live: int) -> int:
+    """Bytes one step must move: predictor, up (and gate) rows of the union
+    (plus bias), down rows of the neurons with a nonzero value, u in, y out."""
+    n_mat_up = 2 if cfg.act == "swiglu" else 1
+    ue = 4 if cfg.wtype == "f32" else 2
+    bias = 4 if cfg.act == "relu" else 0
+    return (predictor_bytes(cfg) + n_up_rows * (n_mat_up * row_bytes(cfg) + bias) + n_live * row_bytes(cfg)
+            + B * cfg.d * ue + B * cfg.d * 4)
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.file, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.file is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        self.file.flush()
+        rows = []
+        with open(self.file.name) as fh:
+            for line in fh:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) >= 9:
+                    rows.append(p)
+        os.unlink(self.file.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max((float(r[3]) for r in rows if r[3].replace(".", "").isdigit()), default=None)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle leg
+
+def oracle_run(layer_host: inputs.LayerTensors, cfg, u_host: torch.Tensor, seconds: float, max_steps: int):
+    """Time the oracle (as it stands, one host thread) on whole tokens until the
+    time budget is spent.  Returns (steps, seconds, bytes)."""
+    import oracle
+    L = oracle.Layer(**layer_host.host_arrays())
+    n, t_tot, b_tot = 0, 0.0, 0
+    T = u_host.shape[0]
+    while n < max_steps:
+        u = u_host[n % T].numpy()
+        t0 = time.perf_counter()
+        pr = oracle.predict(L, u)
+        y = oracle.ffn_masked(L, u, pr["idx"])
+        dt = time.perf_counter() - t0
+        union = np.unique(np.concatenate(pr["idx"])) if len(pr["idx"]) else np.array([], np.int64)
+        if cfg.act == "relu":
+            phi = oracle.neuron_phi(L, u)  # untimed bookkeeping of the live rows
+            live = int(np.sum(np.any(phi[:, union] != 0, axis=0))) if len(union) else 0
+        else:
+            live = len(union)
+        t_tot += dt
+        b_tot += step_bytes(cfg, u.shape[0], len(union), live)
+        n += 1
+        if t_tot >= seconds:
+            break
+    return n, t_tot, b_tot
+
+
+# ----------------------------------------------------------------------------- main
+
+def bench_reference(args, world, rank):
+    if rank != 0:
+        return None
+    cfg = inputs.CONFIGS[args.config]
+    lt = inputs.make_layer(cfg, 0, seed=1000, device="cuda" if torch.cuda.is_available() else "cpu").to("cpu")
+    toks = torch.stack([inputs.layer_input(cfg, inputs.make_tokens(cfg, t, args.batch, seed=1000))
+                        for t in range(args.tokens)])
+    oracle_run(lt, cfg, toks, 0.0, max(1, min(args.warmup, 1)))  # warm-up (page-in)
+    n, sec, nbytes = oracle_run(lt, cfg, toks, args.ref_seconds, args.steps)
+    v = nbytes / sec / 1e9
+    line = {"metric": "sparse-FFN achieved HBM GB/s of touched rows (batch-1 decode)", "value": v, "unit": "GB/s",
+            "impl": "reference", "n_gpus": args.gpus, "steps": n, "warmup": 1, "ms_per_step": sec / n * 1e3,
+            "us_per_layer": sec / n * 1e6, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{cfg.name} single FFN layer d={cfg.d} f={cfg.f} r={cfg.r} {cfg.wtype} "
+                                   f"batch {args.batch}", "batch": args.batch},
+            "cpu_baseline": {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{n} whole tokens of replica 0 (time-bounded at {args.ref_seconds:.0f} s)"},
+            "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    return line
+
+
+def bench_ours(args, world, rank, local):
+    from activation_sparse_decode_gemv_b200 import binding as pb
+    assert torch.cuda.is_available(), "bench.py needs a CUDA device"
+    pb.lib()
+    dev = torch.device("cuda", local)
+    cfg = inputs.CONFIGS[args.config]
+    B, R, T = args.batch, args.replicas, args.tokens
+    seed = 1000 + rank
+    layers = [inputs.make_layer(cfg, r, seed=seed, device=dev) for r in range(R)]
+    handles = [pb.FfnLayer.from_tensors(lt) for lt in layers]
+    ws = pb.make_workspace(handles, B, dev)
+    toks_host = torch.stack([inputs.layer_input(cfg, inputs.make_tokens(cfg, t, B, seed=seed)) for t in range(T)])
+    toks = toks_host.to(dev)
+    y = torch.zeros((B, cfg.d), device=dev)
+    stream = torch.cuda.Stream(dev)
+
+    # bytes of every (replica, token) pair, from the library's own sets (untimed)
+    pair_bytes = {}
+    idx = torch.empty((B, cfg.f), dtype=torch.int32, device=dev)
+    cnt = torch.empty((B,), dtype=torch.int32, device=dev)
+    for r in range(R):
+        lt = layers[r]
+        for t in range(T):
+            pb.pi_decode_ffn(handles[r], toks[t], y, ws, idx=idx, count=cnt, flags=args.flags)
+            torch.cuda.synchronize()
+            c = cnt.cpu().tolist()
+            sets = [idx[b, :c[b]].long() for b in range(B)]
+            union = torch.unique(torch.cat(sets)) if sum(c) else torch.empty(0, dtype=torch.long, device=dev)
+            if cfg.act == "relu" and len(union):
+                W = lt.w_up.index_select(0, union).float()
+                pre = toks[t].float() @ W.T + lt.b_up[union]
+                member = torch.zeros((B, len(union)), dtype=torch.bool, device=dev)
+                for b in range(B):
+                    member[b] = torch.isin(union, sets[b])
+                live = int(((pre > 0) & member).any(0).sum())
+            else:
+                live = len(union)
+            pair_bytes[(r, t)] = step_bytes(cfg, B, len(union), live)
+    assert pb.pi_get_device_status(ws) == 0
+
+    # graphs: one of S = lcm(R, T) steps, plus single-step graphs for a remainder
+    S = int(np.lcm(R, T))
+    sched = [(j % R, j % T) for j in range(S)]
+
+    def step(j):
+        r, t = sched[j]
+        pb.pi_decode_ffn(handles[r], toks[t], y, ws, flags=args.flags, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for j in range(S):  # eager warm-up before capture
+            step(j)
+    stream.synchronize()
+    big = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(big, stream=stream):
+        for j in range(S):
+            step(j)
+    singles = []
+    for j in range(S):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step(j)
+        singles.append(g)
+
+    def run(nsteps):
+        with torch.cuda.stream(stream):
+            for _ in range(nsteps // S):
+                big.replay()
+            for j in range(nsteps % S):
+                singles[j].replay()
+
+    run(args.warmup)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        run(args.steps)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    sec = ev0.elapsed_time(ev1) / 1e3
+    assert pb.pi_get_device_status(ws) == 0
+    nbytes = sum(pair_bytes[sched[j % S]] for j in range(args.steps))
+    gbs, tmax = aggregate(nbytes, sec, world)
+    us_layer = tmax / args.steps * 1e6
+
+    # end to end through the public call: pinned host token -> device, decode, y -> pinned host
+    h_in = toks_host.pin_memory()
+    h_out = torch.empty((args.e2e_steps, B, cfg.d), dtype=torch.float32).pin_memory()
+    u_dev = torch.empty_like(toks[0])
+    n_e2e = args.e2e_steps
+    with torch.cuda.stream(stream):
+        for j in range(min(n_e2e, 64)):  # warm-up
+            r, t = sched[j % S]
+            u_dev.copy_(h_in[t], non_blocking=True)
+            pb.pi_decode_ffn(handles[r], u_dev, y, ws, flags=args.flags, stream=stream)
+            h_out[j].copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for j in range(n_e2e):
+            r, t = sched[j % S]
+            u_dev.copy_(h_in[t], non_blocking=True)
+            pb.pi_decode_ffn(handles[r], u_dev, y, ws, flags=args.flags, stream=stream)
+            h_out[j].copy_(y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_sec = e0.elapsed_time(e1) / 1e3
+    e2e_bytes = sum(pair_bytes[sched[j % S]] for j in range(n_e2e))
+    e2e_gbs, _ = aggregate(e2e_bytes, e2e_sec, world)
+
+    peaks = {}
+    pp = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(pp):
+        peaks = json.load(open(pp))
+    peak = peaks.get("hbm_gbs", 6650.0)
+    per_gpu = gbs / world
+    line = {
+        "metric": "sparse-FFN achieved HBM GB/s of touched rows (batch-1 decode)",
+        "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": tmax / args.steps * 1e3, "us_per_layer": us_layer,
+        "ffn_layer_tokens_per_s": B * args.steps / tmax * world,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "weights": cfg.wtype, "data": "synthetic",
+        "config": {"workload": f"{cfg.name}: single FFN layer d={cfg.d} f={cfg.f} r={cfg.r} {cfg.act} "
+                               f"{cfg.wtype} weights, batch {B}, mean firing rate {cfg.mean_p}",
+                   "batch": B, "d_model": cfg.d, "d_ffn": cfg.f, "rank": cfg.r, "replicas": R, "tokens": T,
+                   "l2": f"{R} rotating seeded replicas ({sum(l.nbytes() for l in layers) / 1e9:.1f} GB) > L2",
+                   "bytes_per_step": nbytes / args.steps, "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "hbm", "achieved": per_gpu, "peak": peak, "unit": "GB/s", "frac": per_gpu / peak,
+                     "traffic": None, "kernel": "whole decode step (5 kernels)",
+                     "peak_source": "measured" if "hbm_gbs" in peaks else "fallback"},
+        "e2e": {"value": e2e_gbs, "unit": "GB/s", "h2d_bytes_per_step": int(toks[0].numel() * toks.element_size()),
+                "d2h_bytes_per_step": int(y.numel() * 4), "steps": n_e2e,
+                "us_per_layer": e2e_sec / n_e2e * 1e6},
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n, csec, cbytes = oracle_run(layers[0].to("cpu"), cfg, toks_host, args.cpu_seconds, 10 ** 9)
+        line["cpu_baseline"] = {"value": cbytes / csec / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                                "sample": f"{n} whole tokens of replica 0, one host thread",
+                                "us_per_layer": csec / n * 1e6}
+    return line
+
+
+def main(argv=None):
+    args = parse(argv)
+    world, rank, local = dist_init()
+    try:
+        line = bench_reference(args, world, rank) if args.impl == "reference" else bench_ours(args, world, rank, local)
+        if rank == 0 and line is not None:
+            s = json.dumps(line)
+            print(s, flush=True)
+            if args.json_out:
+                with open(args.json_out, "w") as fh:
+                    fh.write(s + "\n")
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
