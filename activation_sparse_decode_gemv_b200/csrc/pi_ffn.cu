@@ -9,6 +9,7 @@
 #include <new>
 
 #include "pi_ffn.h"
+#include "pi_fused.cuh"
 #include "pi_kernels.cuh"
 
 struct pi_ffn {
@@ -67,6 +68,7 @@ struct Ws {
   char *base;
   int *status() const { return reinterpret_cast<int *>(base); }
   int32_t *ucount() const { return reinterpret_cast<int32_t *>(base) + 1; }
+  unsigned *grid_bar() const { return reinterpret_cast<unsigned *>(base) + 2; }
   float *h() const { return reinterpret_cast<float *>(base + L.h); }
   __half *u() const { return reinterpret_cast<__half *>(base + L.u); }
   uint32_t *mask() const { return reinterpret_cast<uint32_t *>(base + L.mask); }
@@ -286,9 +288,103 @@ pi_status run_ffn(const pi_ffn *h, const void *u, int B, float *out, int accumul
   }
   PI_CUDA(e);
   const int n_elem = B * D.d_model;
-  PI_CUDA(launch(pi::reduce_kernel, dim3(cdiv(n_elem, 256)), dim3(256), st, (const float *)w.partial(), w.L.G,
-                 (const int32_t *)w.ucount(), (const int32_t *)w.uprefix(), a.hot_dense, h->H, n_elem, out, accumulate));
+  PI_CUDA(launch(pi::reduce_kernel, dim3(cdiv(n_elem, 32)), dim3(256), st, (const float *)w.partial(), w.L.G, n_elem,
+                 out, accumulate));
   return PI_OK;
+}
+
+// ---------------------------------------------------------------- fused batch-1 path
+namespace F = pi::fused;
+
+template <int WT, int ACT, int CPT>
+cudaError_t fused_launch(const F::Args &a, int G, cudaStream_t st) {
+  static bool attr_set = false;
+  const size_t smem = sizeof(F::Smem) + 1024;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(F::decode_fused_kernel<WT, ACT, CPT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    int nb = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, F::decode_fused_kernel<WT, ACT, CPT>, F::kThreads, smem);
+    if (e != cudaSuccess) return e;
+    if (nb < 1) return cudaErrorInvalidConfiguration;
+    attr_set = true;
+  }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(G);
+  cfg.blockDim = dim3(F::kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeCooperative;
+  at[0].val.cooperative = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, F::decode_fused_kernel<WT, ACT, CPT>, a);
+}
+
+// The fused kernel covers batch 1 with fp16 or int4 weights, an fp16
+// predictor of rank <= 1024, and one neuron's rows fitting one 32 KB slot.
+bool fused_ok(const pi_ffn *h, int B, int G) {
+  const pi_ffn_desc &D = h->d;
+  if (B != 1 || D.ptype != PI_W_F16 || D.rank > 1024) return false;
+  if (D.wtype == PI_W_F16) {
+    if (D.d_model > 8192) return false;
+  } else if (D.wtype == PI_W_INT4G32) {
+    if (D.d_model > 8192 || D.d_model % 256) return false;
+  } else {
+    return false;
+  }
+  const long rb = D.wtype == PI_W_F16 ? 2L * D.d_model : D.d_model / 2;
+  const long sb = D.wtype == PI_W_INT4G32 ? D.d_model / 16 : 0;
+  const int nmat = D.act == PI_ACT_SWIGLU ? 3 : 2;
+  if (nmat * (rb + sb) > F::kSlotBytes) return false;
+  const int ntiles = (D.d_ffn + F::kTN - 1) / F::kTN;
+  return ntiles / G + 1 <= F::kMaxOwnTiles;
+}
+
+pi_status run_fused(const pi_ffn *h, const void *in, float *out, int stack, int accumulate, int32_t *idx,
+                    int32_t *count, unsigned flags, const Ws &w, cudaStream_t st) {
+  const pi_ffn_desc &D = h->d;
+  F::Args a{};
+  a.w_up = D.w_up;
+  a.w_gate = D.w_gate;
+  a.w_down_t = D.w_down_t;
+  a.s_up = reinterpret_cast<const __half *>(D.s_up);
+  a.s_gate = reinterpret_cast<const __half *>(D.s_gate);
+  a.s_down_t = reinterpret_cast<const __half *>(D.s_down_t);
+  a.b_up = D.b_up;
+  a.p1 = reinterpret_cast<const __half *>(D.p1);
+  a.p2 = reinterpret_cast<const __half *>(D.p2);
+  a.p_bias = D.p_bias;
+  a.in = in;
+  a.out = out;
+  a.d = D.d_model;
+  a.f = D.d_ffn;
+  a.r = D.rank;
+  a.stack = stack;
+  a.accumulate = accumulate;
+  a.H = want_dense(h, 1, flags) ? h->H : 0;
+  a.h = w.h();
+  a.partial = w.partial();
+  a.mask16 = reinterpret_cast<uint16_t *>(w.mask());
+  a.bar = w.grid_bar();
+  a.status = w.status();
+  a.idx = idx;
+  a.count = count;
+  cudaError_t e;
+  const bool relu = D.act == PI_ACT_RELU;
+  const int G = w.L.G;
+  if (D.wtype == PI_W_F16) {
+    if (D.d_model <= 2 * F::kConsumers * 8)
+      e = relu ? fused_launch<pi::W_F16, pi::ACT_RELU, 2>(a, G, st) : fused_launch<pi::W_F16, pi::ACT_SWIGLU, 2>(a, G, st);
+    else
+      e = relu ? fused_launch<pi::W_F16, pi::ACT_RELU, 4>(a, G, st) : fused_launch<pi::W_F16, pi::ACT_SWIGLU, 4>(a, G, st);
+  } else {
+    e = relu ? fused_launch<pi::W_INT4, pi::ACT_RELU, 2>(a, G, st)
+             : fused_launch<pi::W_INT4, pi::ACT_SWIGLU, 2>(a, G, st);
+  }
+  return e == cudaSuccess ? PI_OK : PI_ERR_CUDA;
 }
 
 pi_status check_call(const pi_ffn *h, int B) {
@@ -401,8 +497,10 @@ pi_status pi_decode_ffn(pi_ffn_t h, const void *u, int B, float *y, int32_t *idx
   const pi_ffn *L[1] = {h};
   if ((s = get_ws(L, 1, B, ws, ws_bytes, &w)) != PI_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
+  const int acc = (flags & PI_FFN_ACCUMULATE) ? 1 : 0;
+  if (fused_ok(h, B, w.L.G)) return run_fused(h, u, y, 0, acc, idx, count, flags, w, st);
   if ((s = run_predict(h, u, B, idx, h->d.d_ffn, count, w, st)) != PI_OK) return s;
-  return run_ffn(h, u, B, y, (flags & PI_FFN_ACCUMULATE) ? 1 : 0, flags, w, st);
+  return run_ffn(h, u, B, y, acc, flags, w, st);
 }
 
 pi_status pi_decode_ffn_stack(const pi_ffn_t *layers, int L, float *x, int B, int32_t *idx_trace,
@@ -426,9 +524,13 @@ pi_status pi_decode_ffn_stack(const pi_ffn_t *layers, int L, float *x, int B, in
   cudaStream_t st = (cudaStream_t)stream;
   const int d = layers[0]->d.d_model;
   for (int l = 0; l < L; ++l) {
-    PI_CUDA(launch(pi::rmsnorm_kernel, dim3(B), dim3(256), st, (const float *)x, d, w.u()));
     int32_t *idx = idx_trace ? idx_trace + (size_t)l * B * fmax : nullptr;
     int32_t *cnt = count_trace ? count_trace + (size_t)l * B : nullptr;
+    if (fused_ok(layers[l], B, w.L.G)) {
+      if ((s = run_fused(layers[l], x, x, 1, 0, idx, cnt, flags, w, st)) != PI_OK) return s;
+      continue;
+    }
+    PI_CUDA(launch(pi::rmsnorm_kernel, dim3(B), dim3(256), st, (const float *)x, d, w.u()));
     if ((s = run_predict(layers[l], w.u(), B, idx, fmax, cnt, w, st)) != PI_OK) return s;
     if ((s = run_ffn(layers[l], w.u(), B, x, 1, flags, w, st)) != PI_OK) return s;
   }

@@ -390,7 +390,6 @@ __global__ void __launch_bounds__(512) ffn_gather_kernel(FfnArgs a) {
   pdl_launch_dependents();
   const int V = virtual_len(a.ucount, a.uprefix, a.hot_dense, a.H);
   const int pb = chunk_begin(c, V, G), pe = chunk_begin(c + 1, V, G);
-  if (pb >= pe) return;
   const int ngroups = d / 8;
   const int upre_h = a.hot_dense ? a.uprefix[a.H >> 5] : 0;
 
@@ -504,21 +503,39 @@ __global__ void __launch_bounds__(512) ffn_gather_kernel(FfnArgs a) {
 }
 
 // ============================================================== reduction
-// out[e] (= or +=) sum over CTAs c with a non-empty range of partial[c][e],
-// in increasing c: deterministic, no atomics.
+// out[e] (= or +=) sum over all CTAs c of partial[c][e] (CTAs without neurons
+// wrote zeros).  A CTA covers 32 consecutive elements; thread (e, g) sums the
+// partials c = g, g + 8, ... in increasing c, then the 8 group sums are added
+// in increasing g: a fixed order, so the result is deterministic, and no
+// atomics are used.
 __global__ void __launch_bounds__(256)
-    reduce_kernel(const float *__restrict__ partial, int G, const int32_t *__restrict__ ucount,
-                  const int32_t *__restrict__ uprefix, int hot_dense, int H, int n_elem, float *__restrict__ out,
-                  int accumulate) {
+    reduce_kernel(const float *__restrict__ partial, int G, int n_elem, float *__restrict__ out, int accumulate) {
+  __shared__ float s_part[8][33];
   pdl_wait();
   pdl_launch_dependents();
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= n_elem) return;
-  const int V = virtual_len(ucount, uprefix, hot_dense, H);
+  const int el = threadIdx.x & 31, g = threadIdx.x >> 5;
+  const int e = blockIdx.x * 32 + el;
   float s = 0.f;
-  for (int c = 0; c < G; ++c)
-    if (chunk_begin(c, V, G) < chunk_begin(c + 1, V, G)) s += partial[(size_t)c * n_elem + e];
-  out[e] = accumulate ? out[e] + s : s;
+  if (e < n_elem) {
+    int c = g;
+    for (; c + 24 < G; c += 32) {
+      const float a0 = partial[(size_t)c * n_elem + e], a1 = partial[(size_t)(c + 8) * n_elem + e];
+      const float a2 = partial[(size_t)(c + 16) * n_elem + e], a3 = partial[(size_t)(c + 24) * n_elem + e];
+      s += a0;
+      s += a1;
+      s += a2;
+      s += a3;
+    }
+    for (; c < G; c += 8) s += partial[(size_t)c * n_elem + e];
+  }
+  s_part[g][el] = s;
+  __syncthreads();
+  if (g == 0 && e < n_elem) {
+    float t = s_part[0][el];
+#pragma unroll
+    for (int k = 1; k < 8; ++k) t += s_part[k][el];
+    out[e] = accumulate ? out[e] + t : t;
+  }
 }
 
 }  // namespace pi

@@ -38,7 +38,11 @@ import torch
 
 from activation_sparse_decode_gemv_b200 import inputs
 
-KERNELS_PER_STEP = 5  # pred_h, pred_s, compact, gather, reduce
+def kernels_per_step(cfg, B):
+    """Launches of the library's kernels per decode step: batch 1 with fp16 /
+    int4 weights runs as one persistent fused kernel; otherwise five kernels
+    (predictor stage 1, stage 2, compaction, gather, reduction)."""
+    return 1 if (B == 1 and cfg.wtype != "f32" and cfg.r <= 1024 and cfg.d <= 8192) else 5
 
 
 def parse(argv=None):
@@ -377,12 +381,14 @@ def bench_ours(args, world, rank, local):
                    "l2": f"{R} rotating seeded replicas ({sum(l.nbytes() for l in layers) / 1e9:.1f} GB) > L2",
                    "bytes_per_step": nbytes / args.steps, "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm", "achieved": per_gpu, "peak": peak, "unit": "GB/s", "frac": per_gpu / peak,
-                     "traffic": None, "kernel": "whole decode step (5 kernels)",
+                     "traffic": None,
+                     "kernel": ("decode_fused_kernel (the whole step is one launch)" if kernels_per_step(cfg, B) == 1
+                                else "whole decode step (5 kernels)"),
                      "peak_source": "measured" if "hbm_gbs" in peaks else "fallback"},
         "e2e": {"value": e2e_gbs, "unit": "GB/s", "h2d_bytes_per_step": int(toks[0].numel() * toks.element_size()),
                 "d2h_bytes_per_step": int(y.numel() * 4), "steps": n_e2e,
                 "us_per_layer": e2e_sec / n_e2e * 1e6},
-        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "gpu_launches": kernels_per_step(cfg, B) * args.steps,
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -148,10 +148,13 @@ int or_dequant_row(int wtype, int d, const void *w, const uint16_t *sc, long row
  *
  * Band: an fp32 evaluation of s differs from this double one by rounding.
  * The band is 16 * 2^-24 * (sqrt(r) sum_j |P2_ij h_j|
- *                           + sqrt(d) sum_j |P2_ij| sum_k |P1_jk u_k|
- *                           + |bias_i|),
+ *                           + sqrt(d) sqrt(sum_j (P2_ij a_j)^2)
+ *                           + |bias_i|),   a_j = sum_k |P1_jk u_k|,
  * a probabilistic rounding-error bound in the style of Higham & Mary
- * (SIAM J. Sci. Comput. 41(5), 2019) with a safety factor of 16.  Neurons
+ * (SIAM J. Sci. Comput. 41(5), 2019) with a safety factor of 16: the error
+ * of a length-n fp32 sum is at most ~sqrt(n) 2^-24 times the sum of the
+ * absolute terms, and the independent errors of the r stage-1 sums h_j reach
+ * s_i through the weights P2_ij, so they combine in quadrature.  Neurons
  * with |s_i| <= band_i may be classified either way by an fp32 evaluation. */
 int or_predict(int d, int f, int r, int ptype, const void *p1, const void *p2, const float *bias,
                int utype, const void *u, int B, double *h_out, double *s_out, double *band_out,
@@ -185,13 +188,13 @@ int or_predict(int d, int f, int r, int ptype, const void *p1, const void *p2, c
         double p = w_elem(p2, NULL, ptype, r, i, j);
         acc += p * h[j];
         t1 += fabs(p * h[j]);
-        t2 += fabs(p) * habs[j];
+        t2 += (p * habs[j]) * (p * habs[j]);
       }
       double s = acc + (double)bias[i];
       if (s_out) s_out[(long)b * f + i] = s;
       if (band_out)
         band_out[(long)b * f + i] =
-            16.0 * ldexp(1.0, -24) * (sqrt((double)r) * t1 + sqrt((double)d) * t2 + fabs((double)bias[i]));
+            16.0 * ldexp(1.0, -24) * (sqrt((double)r) * t1 + sqrt((double)d) * sqrt(t2) + fabs((double)bias[i]));
       if (s > 0.0) idx[(long)b * f + n++] = i;
     }
     count[b] = n;
