@@ -299,7 +299,7 @@ namespace F = pi::fused;
 template <int WT, int ACT, int CPT>
 cudaError_t fused_launch(const F::Args &a, int G, cudaStream_t st) {
   static bool attr_set = false;
-  const size_t smem = sizeof(F::Smem) + 1024;
+  const size_t smem = sizeof(F::Smem);
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(F::decode_fused_kernel<WT, ACT, CPT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
@@ -323,11 +323,11 @@ cudaError_t fused_launch(const F::Args &a, int G, cudaStream_t st) {
   return cudaLaunchKernelEx(&cfg, F::decode_fused_kernel<WT, ACT, CPT>, a);
 }
 
-// The fused kernel covers batch 1 with fp16 or int4 weights, an fp16
-// predictor of rank <= 1024, and one neuron's rows fitting one 32 KB slot.
+// The fused kernel covers batch 1 with fp16 or int4 weights, d <= 8192, an
+// fp16 predictor of rank <= 1024, and one neuron's rows fitting one slot.
 bool fused_ok(const pi_ffn *h, int B, int G) {
   const pi_ffn_desc &D = h->d;
-  if (B != 1 || D.ptype != PI_W_F16 || D.rank > 1024) return false;
+  if (B != 1 || D.ptype != PI_W_F16 || D.rank > F::kMaxR || G > 320) return false;
   if (D.wtype == PI_W_F16) {
     if (D.d_model > 8192) return false;
   } else if (D.wtype == PI_W_INT4G32) {
@@ -339,8 +339,8 @@ bool fused_ok(const pi_ffn *h, int B, int G) {
   const long sb = D.wtype == PI_W_INT4G32 ? D.d_model / 16 : 0;
   const int nmat = D.act == PI_ACT_SWIGLU ? 3 : 2;
   if (nmat * (rb + sb) > F::kSlotBytes) return false;
-  const int ntiles = (D.d_ffn + F::kTN - 1) / F::kTN;
-  return ntiles / G + 1 <= F::kMaxOwnTiles;
+  const int per_cta = (D.d_ffn + G - 1) / G;  // neurons dealt to one CTA
+  return (per_cta + F::kTN - 1) / F::kTN <= F::kMaxOwnTiles;
 }
 
 pi_status run_fused(const pi_ffn *h, const void *in, float *out, int stack, int accumulate, int32_t *idx,
@@ -367,7 +367,7 @@ pi_status run_fused(const pi_ffn *h, const void *in, float *out, int stack, int 
   a.H = want_dense(h, 1, flags) ? h->H : 0;
   a.h = w.h();
   a.partial = w.partial();
-  a.mask16 = reinterpret_cast<uint16_t *>(w.mask());
+  a.mask32 = w.mask();
   a.bar = w.grid_bar();
   a.status = w.status();
   a.idx = idx;

@@ -4,28 +4,35 @@
 // read the rows of the active neurons directly).
 //
 // Grid: one CTA per SM, launched cooperatively (all CTAs co-resident).
-// Block: 8 consumer warps + 1 producer warp.  The producer streams work
-// items into a ring of 6 x 32 KB shared-memory slots with cp.async.bulk (TMA
-// bulk copies) and mbarrier transaction counts; consumers process the slots in
+// Block: 8 consumer warps + 1 producer warp.  The producer streams work items
+// into a ring of 3 x 64 KB shared-memory slots with cp.async.bulk (TMA bulk
+// copies) and mbarrier transaction counts; consumers process the slots in
 // order:
-//   P1 item     rows of P1 owned by this CTA -> its slice of h = P1 u
+//   P1 item     up to 8 rows of P1 owned by this CTA -> its slice of h = P1 u
 //               (then a grid-wide barrier publishes all of h)
-//   P2 tile     16 predictor rows -> s = P2 h + bias, fire iff s > 0; the
-//               tile's active ids go to an in-CTA queue the producer reads
-//   GATHER      up (+gate) and down rows of 1-4 active neurons: dot with u,
-//               activation, then y += a * W2T_i into per-thread registers
+//   P2 tile     32 predictor rows -> s = P2 h + bias, fire iff s > 0.  Warps
+//               record the fired bits with shared-memory atomics and release
+//               the slot without a block barrier.
+//   GATHER      up (+gate) and down rows of 1-4 neurons: dot with u,
+//               activation, then y += a * W2T_i in per-thread registers
 //   DONE        end of the stream
-// The producer issues P2 tiles while the consumers wait on the h barrier,
-// so the memory system keeps streaming, and issues a tile's gather rows as
-// soon as its actives are published.  Tiles of 16 neurons are dealt round
-// robin to the CTAs; in dense hot-prefix mode the prefix tiles' rows are
-// issued with the tile, without waiting for the predictor.
+// The producer "harvests" a tile when its slot's empty barrier completes
+// (every consumer warp is done with it), appends the fired ids to its list
+// and issues their gather rows; it keeps issuing P2 tiles meanwhile, and it
+// prefetches tiles while the consumers wait on the h barrier.  Neurons are
+// dealt round robin to the CTAs (neuron i to CTA i mod G), so every CTA gets
+// the same mix of hot and cold neurons; CTA c's k-th tile holds its own
+// neurons c + (32k + q) G, q < 32.  In dense hot-prefix mode the rows of a
+// tile's prefix neurons are issued right after the tile, without waiting
+// for its bits.
 // After the stream every CTA writes its fp32 partial of y; a second grid
 // barrier; each CTA then sums a column slice over all partials in CTA order
 // (deterministic, no atomics) and writes y (or adds it to the residual x).
 // Every wait is bounded (about 2 s); on expiry the kernel records
 // PI_ERR_TIMEOUT in the workspace status word and completes.
 #pragma once
+
+#include <cstddef>
 
 #include "pi_device.cuh"
 
@@ -35,12 +42,14 @@ namespace fused {
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kThreads = kConsumers + 32;
-constexpr int kSlots = 6;
-constexpr int kSlotBytes = 32768;
-constexpr int kTN = 16;          // neurons per predictor tile
-constexpr int kMaxGN = 4;        // neurons per gather item
-constexpr int kActCap = 2048;    // own active-queue capacity (>= own neurons)
-constexpr int kMaxOwnTiles = 128;
+constexpr int kSlots = 3;
+constexpr int kSlotBytes = 65536;
+constexpr int kTN = 32;                      // neurons per predictor tile
+constexpr int kMaxGN = 4;                    // neurons per gather item
+constexpr int kMaxOwnTiles = 32;             // neurons per CTA <= 32 * 32
+constexpr int kActCap = kMaxOwnTiles * kTN;  // capacity of the active-id list
+constexpr int kMaxR = 1024;                  // predictor rank
+constexpr int kMaxP1Rows = 8;                // P1 rows per item
 constexpr unsigned long long kWaitNs = 2000000000ull;
 
 enum ItemType : int { IT_P1 = 0, IT_P2 = 1, IT_GATHER = 2, IT_DONE = 3 };
@@ -55,17 +64,24 @@ struct Smem {
   SlotMeta meta[kSlots];
   unsigned long long full[kSlots];
   unsigned long long empty[kSlots];
-  unsigned tbits[kSlots];
-  int act[kActCap];
-  uint16_t own_bits[kMaxOwnTiles];
+  unsigned tbits[kSlots];              // fired bits of the tile in a slot
+  unsigned own_bits[kMaxOwnTiles];     // fired bits of this CTA's tiles
+  int act[kActCap];                    // fired ids (index mode), producer-owned
+  int tile_item[kMaxOwnTiles];         // item number each own tile was issued as
+  float own_pbias[kMaxOwnTiles][kTN];  // predictor bias of this CTA's neurons
+  float own_bup[kMaxOwnTiles][kTN];    // ReLU bias b1 of this CTA's neurons
+  alignas(16) float h_s[kMaxR];  // written with 16-byte vector stores
   float red[2][kConsumerWarps][2 * kMaxGN];
   double dred[kConsumerWarps];
   float fin[kConsumerWarps][33];
   int iscan[kConsumerWarps];
-  volatile int act_tail;
-  volatile int tiles_done;
   volatile int abort_flag;
 };
+
+static_assert(offsetof(Smem, ring) == 0, "ring slots must start the shared block");
+static_assert(kSlotBytes % 16 == 0, "bulk copies need 16-byte aligned slots");
+static_assert(offsetof(Smem, h_s) % 16 == 0, "h_s is accessed with 16-byte vectors");
+static_assert(sizeof(Smem) <= 227 * 1024, "shared memory per block");
 
 struct Args {
   const void *w_up, *w_gate, *w_down_t;
@@ -78,10 +94,10 @@ struct Args {
   int d, f, r;
   int stack;       // input is the residual x: RMS-normalise it, and add y into it
   int accumulate;  // y += (non-stack)
-  int H;           // dense hot-prefix neurons (multiple of 16); 0 = index mode
+  int H;           // dense hot-prefix neurons [0, H); 0 = index mode
   float *h;        // workspace [r]
   float *partial;  // workspace [G x d]
-  uint16_t *mask16;  // workspace [ceil(f/16)], written when idx != nullptr
+  unsigned *mask32;  // workspace [ceil(f/32)] fired bits of neurons 32w..32w+31, when idx or count != nullptr
   unsigned *bar;     // workspace grid-barrier word
   int *status;
   int32_t *idx;    // optional ascending active ids [f]
@@ -104,10 +120,21 @@ PI_DEV void mbar_arrive_tx(unsigned long long *b, unsigned tx) {
 PI_DEV void mbar_arrive(unsigned long long *b) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
 }
-PI_DEV bool mbar_try(unsigned long long *b, unsigned parity) {
+// try_wait with a suspend-time hint: the thread is parked until the phase
+// completes or the hint (ns) elapses, instead of spinning on the barrier
+PI_DEV bool mbar_try(unsigned long long *b, unsigned parity, unsigned hint_ns) {
   unsigned ok;
   asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(b)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+PI_DEV bool mbar_test(unsigned long long *b, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(ok)
       : "r"(smem_u32(b)), "r"(parity)
       : "memory");
@@ -115,11 +142,10 @@ PI_DEV bool mbar_try(unsigned long long *b, unsigned parity) {
 }
 // bounded wait; false on timeout (status recorded)
 PI_DEV bool mbar_wait(unsigned long long *b, unsigned parity, int *status) {
-  if (mbar_try(b, parity)) return true;
+  if (mbar_test(b, parity)) return true;
   const unsigned long long t0 = globaltimer();
   for (;;) {
-    for (int k = 0; k < 64; ++k)
-      if (mbar_try(b, parity)) return true;
+    if (mbar_try(b, parity, 20000u)) return true;
     if (globaltimer() - t0 > kWaitNs) {
       set_status(status, kStatusTimeout);
       return false;
@@ -170,28 +196,78 @@ template <> struct Cols<W_INT4> {
   static constexpr int EC = 16;
 };
 
-PI_DEV float dot8_h(const uint4 &w, const float *u) {
-  float wf[8];
-  h8_to_f8(w, wf);
-  float a = wf[0] * u[0];
-#pragma unroll
-  for (int k = 1; k < 8; ++k) a = fmaf(wf[k], u[k], a);
-  return a;
+// dot of 8 fp16 weights with 8 fp32 values as two independent chains
+PI_DEV float dot8_h2(const uint4 &w, const float *u) {
+  const __half2 *hp = reinterpret_cast<const __half2 *>(&w);
+  const float2 a0 = __half22float2(hp[0]), a1 = __half22float2(hp[1]);
+  const float2 a2 = __half22float2(hp[2]), a3 = __half22float2(hp[3]);
+  float x = a0.x * u[0], y = a0.y * u[1];
+  x = fmaf(a1.x, u[2], x);
+  y = fmaf(a1.y, u[3], y);
+  x = fmaf(a2.x, u[4], x);
+  y = fmaf(a2.y, u[5], y);
+  x = fmaf(a3.x, u[6], x);
+  y = fmaf(a3.y, u[7], y);
+  return x + y;
 }
-// 16 int4 values (one 8-byte word pair) times u, without the group scale
+// 16 int4 values (one 8-byte word pair) times u, without the group scale,
+// as two independent chains
 PI_DEV float dot16_q(uint2 w, const float *u) {
-  float a = 0.f;
-  const uint32_t ws[2] = {w.x, w.y};
+  float x = 0.f, y = 0.f;
 #pragma unroll
-  for (int j = 0; j < 2; ++j) {
-#pragma unroll
-    for (int k = 0; k < 8; ++k) a = fmaf((float)((int)((ws[j] >> (4 * k)) & 15u) - 8), u[8 * j + k], a);
+  for (int k = 0; k < 8; ++k) {
+    x = fmaf((float)((int)((w.x >> (4 * k)) & 15u) - 8), u[k], x);
+    y = fmaf((float)((int)((w.y >> (4 * k)) & 15u) - 8), u[8 + k], y);
   }
-  return a;
+  return x + y;
 }
 
-// P1 rows per work item (one slot, at most 4 so that a thread keeps 4 sums)
-PI_DEV int p1_rows_per_item(int d) { return min(4, kSlotBytes / (d * 2)); }
+// 8 fp16 weights times 8 fp16 inputs (16 B each), accumulated into two fp32
+// chains with the mixed-precision FMA: the product of two fp16 values is exact
+// in fp32, so each step equals fmaf((float)w, (float)u, acc) bit for bit
+PI_DEV void dot8_mixed(const uint4 &w, const uint4 &u, float &x, float &y) {
+  const unsigned ws[4] = {w.x, w.y, w.z, w.w}, us[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    asm("{\n .reg .b16 al, ah, bl, bh;\n mov.b32 {al, ah}, %2;\n mov.b32 {bl, bh}, %3;\n"
+        " fma.rn.f32.f16 %0, al, bl, %0;\n fma.rn.f32.f16 %1, ah, bh, %1;\n}\n"
+        : "+f"(x), "+f"(y)
+        : "r"(ws[k]), "r"(us[k]));
+}
+// the 8 int4 codes of one 32-bit word (element 2k = low nibble of byte k) as
+// four fp16 pairs (q - 8): 0x6400 | q is the fp16 value 1024 + q, and
+// subtracting 1032 is exact
+PI_DEV void q8_to_h2(uint32_t w, uint32_t out[4]) {
+  const __half2 off = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t t = w >> (8 * k);
+    const uint32_t hb = (t & 0xFu) | ((t & 0xF0u) << 12) | 0x64006400u;
+    const __half2 v = __hsub2(*reinterpret_cast<const __half2 *>(&hb), off);
+    out[k] = *reinterpret_cast<const uint32_t *>(&v);
+  }
+}
+// 16 int4 codes (q - 8) times 16 fp16 inputs, without the group scale
+PI_DEV void dot16_q_mixed(const uint2 &w, const uint4 &u0, const uint4 &u1, float &x, float &y) {
+  uint32_t q[8];
+  q8_to_h2(w.x, q);
+  q8_to_h2(w.y, q + 4);
+  dot8_mixed(make_uint4(q[0], q[1], q[2], q[3]), u0, x, y);
+  dot8_mixed(make_uint4(q[4], q[5], q[6], q[7]), u1, x, y);
+}
+
+// sum N independent values across the warp; the N butterflies are
+// interleaved so that their shuffles overlap
+template <int N>
+PI_DEV void warp_sum_n(float (&v)[N]) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+    for (int k = 0; k < N; ++k) v[k] += __shfl_xor_sync(0xffffffffu, v[k], o);
+  }
+}
+
+PI_DEV int p1_rows_per_item(int d) { return min(kMaxP1Rows, kSlotBytes / (d * 2)); }
 
 // bytes of one weight row and of one int4 scale row
 template <int WT>
@@ -227,20 +303,47 @@ struct NeuronLayout {
   }
 };
 
+// neurons of CTA c: i = c + m G, m < own_count; tile k holds m in [32k, 32k + 32)
+PI_DEV int own_count(int f, int c, int G) { return c < f ? (f - 1 - c) / G + 1 : 0; }
+
 // ---------------------------------------------------------------- producer
 template <int WT, int ACT>
 PI_DEV void producer(Smem &S, const Args &a, int c, int G) {
   const int d = a.d, f = a.f, r = a.r;
-  const int ntiles = (f + kTN - 1) / kTN;
-  const int nown = (c < ntiles) ? (ntiles - 1 - c) / G + 1 : 0;
+  const int nn = own_count(f, c, G);
+  const int nown = (nn + kTN - 1) / kTN;
   const int j0 = (int)((long long)c * r / G), j1 = (int)((long long)(c + 1) * r / G);
   const int rpi = p1_rows_per_item(d);
   const NeuronLayout<WT, ACT> NL(d);
   const int GN = min(kMaxGN, kSlotBytes / (int)NL.bytes);
   const unsigned rb = wrow_bytes<WT>(d), sb = srow_bytes<WT>(d);
-  unsigned pn = 0;
+  const bool want_mask = a.idx != nullptr || a.count != nullptr;
+  unsigned pn = 0;       // items issued
+  int k = 0;             // own tiles issued
+  int hk = 0;            // own tiles harvested
+  int act_tail = 0;      // fired ids appended (index mode)
+  int taken = 0;         // fired ids issued as gather items
   bool ok = true;
 
+  // fired bits of own tile hk are final once its slot's empty phase completed
+  auto harvest = [&]() {
+    const int s = S.tile_item[hk] % kSlots;
+    unsigned b = S.tbits[s];
+    while (b) {
+      const int q = __ffs(b) - 1;
+      b &= b - 1u;
+      const int i = c + (hk * kTN + q) * G;
+      if (want_mask) atomicOr(a.mask32 + (i >> 5), 1u << (i & 31));
+      if (i >= a.H) S.act[act_tail++] = i;
+    }
+    ++hk;
+  };
+  auto tile_done = [&](int kk) -> bool {
+    const unsigned it = (unsigned)S.tile_item[kk];
+    return mbar_test(&S.empty[it % kSlots], (it / kSlots) & 1u);
+  };
+  // next slot in ring order; every tile that lived in a slot freed so far is
+  // harvested before its slot is overwritten
   auto acquire = [&](int &s) -> bool {
     s = (int)(pn % kSlots);
     const unsigned par = ((pn / kSlots) & 1u) ^ 1u;
@@ -248,6 +351,7 @@ PI_DEV void producer(Smem &S, const Args &a, int c, int G) {
       S.abort_flag = 1;
       return false;
     }
+    while (hk < k && (unsigned)S.tile_item[hk] + kSlots <= pn) harvest();
     return true;
   };
   auto issue_gather = [&](const int *ids, int n) -> bool {
@@ -290,62 +394,55 @@ PI_DEV void producer(Smem &S, const Args &a, int c, int G) {
     ++pn;
   }
   // 2. predictor tiles and gather rows
-  int k = 0, taken = 0;
-  unsigned long long t0 = 0;
   while (ok) {
-    const int tail = S.act_tail;
-    __threadfence_block();
-    if (taken < tail) {
-      const int n = min(GN, tail - taken);
+    while (hk < k && tile_done(hk)) harvest();
+    if (taken < act_tail) {
+      const int n = min(GN, act_tail - taken);
       ok = issue_gather(&S.act[taken], n);
       taken += n;
-      t0 = 0;
       continue;
     }
     if (k < nown) {
-      const int tile = c + k * G;
-      const int rows = min(kTN, f - tile * kTN);
+      const int rows = min(kTN, nn - k * kTN);
       int s;
       if (!(ok = acquire(s))) break;
       S.meta[s].type = IT_P2;
       S.meta[s].n = rows;
-      S.meta[s].first = tile;
+      S.meta[s].first = k;
       S.tbits[s] = 0u;
-      const unsigned bytes = (unsigned)rows * (unsigned)r * 2u;
-      mbar_arrive_tx(&S.full[s], bytes);
-      bulk_g2s(S.ring[s], a.p2 + (size_t)tile * kTN * r, bytes, &S.full[s]);
+      S.tile_item[k] = (int)pn;
+      const unsigned rbp = (unsigned)r * 2u;
+      mbar_arrive_tx(&S.full[s], (unsigned)rows * rbp);
+      for (int q = 0; q < rows; ++q)
+        bulk_g2s(S.ring[s] + q * rbp, a.p2 + (size_t)(c + (k * kTN + q) * G) * r, rbp, &S.full[s]);
       ++pn;
-      if (tile * kTN < a.H) {  // dense hot prefix: every row of the tile, now
-        int ids[kMaxGN];
-        for (int q = 0; ok && q < rows; q += GN) {
-          const int n = min(GN, rows - q);
-          for (int g = 0; g < n; ++g) ids[g] = tile * kTN + q + g;
-          ok = issue_gather(ids, n);
+      // dense hot prefix: the tile's prefix neurons (the smallest ids), now
+      int ids[kMaxGN], ng = 0;
+      for (int q = 0; ok && q < rows; ++q) {
+        const int i = c + (k * kTN + q) * G;
+        if (i >= a.H) break;
+        ids[ng++] = i;
+        if (ng == GN) {
+          ok = issue_gather(ids, ng);
+          ng = 0;
         }
       }
+      if (ok && ng) ok = issue_gather(ids, ng);
       ++k;
-      t0 = 0;
       continue;
     }
-    if (S.tiles_done == nown) {
-      __threadfence_block();
-      if (S.act_tail == taken) break;
-      continue;
-    }
-    if (S.abort_flag) {
-      ok = false;
-      break;
-    }
-    if (t0 == 0) t0 = globaltimer();
-    if (globaltimer() - t0 > kWaitNs) {
-      set_status(a.status, kStatusTimeout);
+    if (hk == nown) break;  // every tile harvested and every fired id issued
+    // wait for the consumers to finish the oldest unharvested tile
+    const unsigned it = (unsigned)S.tile_item[hk];
+    if (!mbar_wait(&S.empty[it % kSlots], (it / kSlots) & 1u, a.status)) {
       S.abort_flag = 1;
       ok = false;
       break;
     }
-    __nanosleep(32);
+    harvest();
   }
   // 3. end of stream (also after an abort, so consumers stop)
+  __threadfence();  // mask words visible before the consumers' grid barrier
   int s;
   if (acquire(s)) {
     S.meta[s].type = IT_DONE;
@@ -360,23 +457,26 @@ PI_DEV void producer(Smem &S, const Args &a, int c, int G) {
 // CPT: column chunks per consumer thread (d <= CPT * 256 * EC)
 template <int WT, int ACT, int CPT>
 __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Args a) {
-  extern __shared__ uint8_t smem_raw[];
-  Smem &S = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  // indexed directly (no integer round trip) so that every access stays in
+  // the shared state space; bulk copies need only 16-byte alignment
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  Smem &S = *reinterpret_cast<Smem *>(smem_raw);
   constexpr int EC = Cols<WT>::EC;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, c = blockIdx.x;
   const int d = a.d, f = a.f, r = a.r;
+  const int nwords = (f + 31) / 32;
+  const int nn = own_count(f, c, G);
 
   if (tid == 0) {
     for (int s = 0; s < kSlots; ++s) {
       mbar_init(&S.full[s], 1);
       mbar_init(&S.empty[s], kConsumerWarps);
     }
-    S.act_tail = 0;
-    S.tiles_done = 0;
     S.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  for (int k = tid; k < kMaxOwnTiles; k += blockDim.x) S.own_bits[k] = 0u;
   __syncthreads();
 
   if (warp == kConsumerWarps) {
@@ -386,14 +486,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Args a) {
 
   // ------------------------------------------------------------ consumers
   const int nch = d / EC;
-  const int ntiles = (f + kTN - 1) / kTN;
   const int j0 = (int)((long long)c * r / G), j1 = (int)((long long)(c + 1) * r / G);
   const int rpi = p1_rows_per_item(d);
   const int n_p1 = (j1 - j0 + rpi - 1) / rpi;
   const NeuronLayout<WT, ACT> NL(d);
 
-  // FFN input u for the owned columns (fp32 registers)
-  float u[CPT][EC];
+  // FFN input u (fp16) for the owned column chunks, packed; chunks past the
+  // row end hold zeros and read a clamped, valid address (branch-free loops)
+  constexpr int UW = EC / 8;  // uint4 words of u per chunk
+  uint4 uh[CPT][UW];
+  int coff[CPT];  // clamped chunk index
+#pragma unroll
+  for (int q = 0; q < CPT; ++q) coff[q] = min(tid + q * kConsumers, nch - 1);
   if (a.stack) {
     const float *x = reinterpret_cast<const float *>(a.in);
     double ss = 0.0;
@@ -411,24 +515,28 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Args a) {
     const float den = __fsqrt_rn(__fadd_rn(mean, 1e-6f));
 #pragma unroll
     for (int q = 0; q < CPT; ++q) {
-      const int ch = tid + q * kConsumers;
+      const bool valid = tid + q * kConsumers < nch;
 #pragma unroll
-      for (int e = 0; e < EC; ++e)
-        u[q][e] = (ch < nch) ? __half2float(__float2half_rn(__fdiv_rn(x[ch * EC + e], den))) : 0.f;
+      for (int j = 0; j < UW; ++j) {
+        uint32_t wd[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int e = coff[q] * EC + 8 * j + 2 * k;
+          const __half lo = __float2half_rn(__fdiv_rn(x[e], den)), hi = __float2half_rn(__fdiv_rn(x[e + 1], den));
+          wd[k] = valid ? ((uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16)) : 0u;
+        }
+        uh[q][j] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+      }
     }
   } else {
-    const __half *uh = reinterpret_cast<const __half *>(a.in);
+    const __half *uin = reinterpret_cast<const __half *>(a.in);
 #pragma unroll
     for (int q = 0; q < CPT; ++q) {
-      const int ch = tid + q * kConsumers;
+      const bool valid = tid + q * kConsumers < nch;
 #pragma unroll
-      for (int e = 0; e < EC; e += 8) {
-        if (ch < nch) {
-          h8_to_f8(ld_keep16(uh + ch * EC + e), &u[q][e]);
-        } else {
-#pragma unroll
-          for (int k = 0; k < 8; ++k) u[q][e + k] = 0.f;
-        }
+      for (int j = 0; j < UW; ++j) {
+        const uint4 v = ld_keep16(uin + coff[q] * EC + 8 * j);
+        uh[q][j] = valid ? v : make_uint4(0u, 0u, 0u, 0u);
       }
     }
   }
@@ -437,6 +545,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Args a) {
   for (int q = 0; q < CPT; ++q)
 #pragma unroll
     for (int e = 0; e < EC; ++e) y[q][e] = 0.f;
+
+  // biases of this CTA's own neurons c + m G, one round trip
+  for (int m = tid; m < nn; m += kConsumers) {
+    const int i = c + m * G;
+    S.own_pbias[m / kTN][m % kTN] = __ldg(a.p_bias + i);
+    if (ACT == ACT_RELU) S.own_bup[m / kTN][m % kTN] = __ldg(a.b_up + i);
+  }
+  // clear the fired-bit words (CTA c clears words c, c + G, ...); the first
+  // grid barrier orders this before any CTA sets bits
+  if (a.idx != nullptr || a.count != nullptr)
+    for (int w = c + tid * G; w < nwords; w += kConsumers * G) a.mask32[w] = 0u;
 
   unsigned n = 0;   // items consumed
   unsigned nr = 0;  // reductions done (parity of the red buffer)
@@ -455,41 +574,35 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Args a) {
     ++n;
   };
 
-  // ---- P1 items: this CTA's slice of h
+  // ---- P1 items: this CTA's slice of h (rows past the item alias row 0)
   for (int it = 0; it < n_p1 && alive; ++it) {
     int s;
     if (!(alive = wait_full(s))) break;
     const int rows = S.meta[s].n, jf = S.meta[s].first;
-    float part[4];
+    float px[kMaxP1Rows], py[kMaxP1Rows];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) part[q] = 0.f;
+    for (int q = 0; q < kMaxP1Rows; ++q) {
+      px[q] = py[q] = 0.f;
+      const __half *row = reinterpret_cast<const __half *>(S.ring[s]) + (size_t)(q < rows ? q : 0) * d;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      if (q >= rows) break;
-      const __half *row = reinterpret_cast<const __half *>(S.ring[s]) + (size_t)q * d;
-      float acc = 0.f;
+      for (int cq = 0; cq < CPT; ++cq)
 #pragma unroll
-      for (int cq = 0; cq < CPT; ++cq) {
-        const int ch = tid + cq * kConsumers;
-        if (ch < nch) {
-#pragma unroll
-          for (int e = 0; e < EC; e += 8)
-            acc += dot8_h(*reinterpret_cast<const uint4 *>(row + ch * EC + e), &u[cq][e]);
-        }
-      }
-      part[q] = acc;
+        for (int j = 0; j < UW; ++j)
+          dot8_mixed(*reinterpret_cast<const uint4 *>(row + coff[cq] * EC + 8 * j), uh[cq][j], px[q], py[q]);
     }
+    float part[kMaxP1Rows];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) part[q] = warp_sum(part[q]);
+    for (int q = 0; q < kMaxP1Rows; ++q) part[q] = px[q] + py[q];
+    warp_sum_n<kMaxP1Rows>(part);
     const int par = nr & 1;
     if (lane == 0) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) S.red[par][warp][q] = part[q];
+      for (int q = 0; q < kMaxP1Rows; ++q) S.red[par][warp][q] = part[q];
     }
     release(s);
     consumer_sync();
     ++nr;
-    if (tid < rows && tid < 4) {
+    if (tid < rows) {
       float t = 0.f;
 #pragma unroll
       for (int w = 0; w < kConsumerWarps; ++w) t += S.red[par][w][tid];
@@ -502,14 +615,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Args a) {
     if (!grid_barrier(a.bar, G, c, a.status)) S.abort_flag = 1;
   }
   consumer_sync();
-  // predictor columns of this lane: chunks lane + 32 kk (8 fp16 each)
   const int pch = r / 8;
+  for (int e = tid; e < r / 4; e += kConsumers)
+    reinterpret_cast<float4 *>(S.h_s)[e] = __ldcg(reinterpret_cast<const float4 *>(a.h) + e);
+  consumer_sync();
+  // predictor columns of this lane: chunks lane + 32 kk (8 fp16 each)
   float hreg[4][8];
+  int hoff[4];
 #pragma unroll
   for (int kk = 0; kk < 4; ++kk) {
     const int ch = lane + 32 * kk;
+    hoff[kk] = min(ch, pch - 1);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) hreg[kk][e] = (ch < pch) ? ld_cg(a.h + ch * 8 + e) : 0.f;
+    for (int e = 0; e < 8; ++e) hreg[kk][e] = (ch < pch) ? S.h_s[ch * 8 + e] : 0.f;
   }
 
   // ---- main stream
@@ -522,129 +640,148 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Args a) {
       break;
     }
     if (type == IT_P2) {
-      const int tile = S.meta[s].first, rows = S.meta[s].n;
+      // rows warp + 8 q of the tile, two rows at a time
+      const int kl = S.meta[s].first, rows = S.meta[s].n;
+      constexpr int RPW = kTN / kConsumerWarps;
+      unsigned b = 0u;
 #pragma unroll
-      for (int rr = 0; rr < kTN / kConsumerWarps; ++rr) {
-        const int row_i = warp + rr * kConsumerWarps;
-        if (row_i < rows) {
-          const __half *row = reinterpret_cast<const __half *>(S.ring[s]) + (size_t)row_i * r;
-          float acc = 0.f;
+      for (int rp = 0; rp < RPW; rp += 2) {
+        uint4 wv[2][4];
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const int ch = lane + 32 * kk;
-            if (ch < pch) acc += dot8_h(*reinterpret_cast<const uint4 *>(row + ch * 8), hreg[kk]);
-          }
-          acc = warp_sum(acc);
-          const int i = tile * kTN + row_i;
-          if (lane == 0 && acc + __ldg(a.p_bias + i) > 0.f) atomicOr(&S.tbits[s], 1u << row_i);
+        for (int q = 0; q < 2; ++q) {
+          const int row_i = warp + (rp + q) * kConsumerWarps;
+          const __half *row = reinterpret_cast<const __half *>(S.ring[s]) + (size_t)min(row_i, rows - 1) * r;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) wv[q][kk] = *reinterpret_cast<const uint4 *>(row + hoff[kk] * 8);
+        }
+        float sv[2];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          float acc[4];
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) acc[kk] = dot8_h2(wv[q][kk], hreg[kk]);
+          sv[q] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        }
+        warp_sum_n<2>(sv);
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int row_i = warp + (rp + q) * kConsumerWarps;
+          if (row_i < rows && sv[q] + S.own_pbias[kl][row_i] > 0.f) b |= 1u << row_i;
         }
       }
-      consumer_sync();
-      if (tid == 0) {
-        const unsigned bits = S.tbits[s];
-        S.own_bits[(tile - c) / G] = (uint16_t)bits;
-        if (a.idx || a.count) a.mask16[tile] = (uint16_t)bits;
-        if (tile * kTN >= a.H) {
-          int t = S.act_tail;
-          unsigned b = bits;
-          while (b) {
-            const int bit = __ffs(b) - 1;
-            b &= b - 1u;
-            S.act[t++] = tile * kTN + bit;
-          }
-          __threadfence_block();
-          S.act_tail = t;
-        }
-        __threadfence_block();
-        S.tiles_done = S.tiles_done + 1;
+      if (lane == 0 && b) {
+        atomicOr(&S.tbits[s], b);
+        atomicOr(&S.own_bits[kl], b);
       }
       release(s);
       continue;
     }
-    // IT_GATHER
+    // IT_GATHER: neurons past the item alias neuron 0 and get a zero value
     const int ng = S.meta[s].n;
-    float part[kMaxGN][2];
+    const uint8_t *nd[kMaxGN];
 #pragma unroll
-    for (int g = 0; g < kMaxGN; ++g) part[g][0] = part[g][1] = 0.f;
+    for (int g = 0; g < kMaxGN; ++g) nd[g] = S.ring[s] + (g < ng ? g : 0) * NL.bytes;
+    float pu[kMaxGN], pg[kMaxGN];
 #pragma unroll
     for (int g = 0; g < kMaxGN; ++g) {
-      if (g < ng) {
-        const uint8_t *nd = S.ring[s] + g * NL.bytes;
+      float ux = 0.f, uy = 0.f, gx = 0.f, gy = 0.f;
 #pragma unroll
-        for (int cq = 0; cq < CPT; ++cq) {
-          const int ch = tid + cq * kConsumers;
-          if (ch < nch) {
-            if (WT == W_F16) {
-              part[g][0] += dot8_h(*reinterpret_cast<const uint4 *>(nd + NL.up + ch * 16), u[cq]);
-              if (ACT == ACT_SWIGLU)
-                part[g][1] += dot8_h(*reinterpret_cast<const uint4 *>(nd + NL.gate + ch * 16), u[cq]);
-            } else {
-              const float su = __half2float(*reinterpret_cast<const __half *>(nd + NL.sup + (ch >> 1) * 2));
-              part[g][0] = fmaf(su, dot16_q(*reinterpret_cast<const uint2 *>(nd + NL.up + ch * 8), u[cq]), part[g][0]);
-              if (ACT == ACT_SWIGLU) {
-                const float sg = __half2float(*reinterpret_cast<const __half *>(nd + NL.sgate + (ch >> 1) * 2));
-                part[g][1] =
-                    fmaf(sg, dot16_q(*reinterpret_cast<const uint2 *>(nd + NL.gate + ch * 8), u[cq]), part[g][1]);
-              }
-            }
+      for (int cq = 0; cq < CPT; ++cq) {
+        if (WT == W_F16) {
+          dot8_mixed(*reinterpret_cast<const uint4 *>(nd[g] + NL.up + coff[cq] * 16), uh[cq][0], ux, uy);
+          if (ACT == ACT_SWIGLU)
+            dot8_mixed(*reinterpret_cast<const uint4 *>(nd[g] + NL.gate + coff[cq] * 16), uh[cq][0], gx, gy);
+        } else {
+          const float su = __half2float(*reinterpret_cast<const __half *>(nd[g] + NL.sup + (coff[cq] >> 1) * 2));
+          float x = 0.f, yv = 0.f;
+          dot16_q_mixed(*reinterpret_cast<const uint2 *>(nd[g] + NL.up + coff[cq] * 8), uh[cq][0], uh[cq][1], x, yv);
+          ux = fmaf(su, x + yv, ux);
+          if (ACT == ACT_SWIGLU) {
+            const float sg = __half2float(*reinterpret_cast<const __half *>(nd[g] + NL.sgate + (coff[cq] >> 1) * 2));
+            float x2 = 0.f, y2 = 0.f;
+            dot16_q_mixed(*reinterpret_cast<const uint2 *>(nd[g] + NL.gate + coff[cq] * 8), uh[cq][0], uh[cq][1], x2,
+                          y2);
+            gx = fmaf(sg, x2 + y2, gx);
           }
         }
       }
+      pu[g] = ux + uy;
+      pg[g] = gx + gy;
     }
     const int par = nr & 1;
+    {
+      constexpr int NV = (ACT == ACT_SWIGLU) ? 2 * kMaxGN : kMaxGN;
+      float pv[NV];
 #pragma unroll
-    for (int g = 0; g < kMaxGN; ++g) {
-      if (g < ng) {
-        const float v0 = warp_sum(part[g][0]);
-        const float v1 = (ACT == ACT_SWIGLU) ? warp_sum(part[g][1]) : 0.f;
-        if (lane == 0) {
-          S.red[par][warp][2 * g] = v0;
-          S.red[par][warp][2 * g + 1] = v1;
+      for (int g = 0; g < kMaxGN; ++g) {
+        pv[(ACT == ACT_SWIGLU) ? 2 * g : g] = pu[g];
+        if (ACT == ACT_SWIGLU) pv[2 * g + 1] = pg[g];
+      }
+      warp_sum_n<NV>(pv);
+      if (lane == 0) {
+#pragma unroll
+        for (int g = 0; g < kMaxGN; ++g) {
+          S.red[par][warp][2 * g] = pv[(ACT == ACT_SWIGLU) ? 2 * g : g];
+          S.red[par][warp][2 * g + 1] = (ACT == ACT_SWIGLU) ? pv[2 * g + 1] : 0.f;
         }
       }
     }
+    // after this barrier every warp has also finished every earlier item,
+    // so the fired bits of the neurons' tiles are complete
     consumer_sync();
     ++nr;
+    // sum the 8 warps' partials: lane (g, w) = (lane / 8, lane % 8) loads
+    // warp w's partial of neuron g, a 3-step butterfly over the 8 lanes of a
+    // group adds them in a fixed order, and shuffles broadcast the sums
+    float av[kMaxGN];
+    {
+      static_assert(kMaxGN * kConsumerWarps == 32, "one lane per (neuron, warp)");
+      float vu = S.red[par][lane & 7][2 * (lane >> 3)];
+      float vg = (ACT == ACT_SWIGLU) ? S.red[par][lane & 7][2 * (lane >> 3) + 1] : 0.f;
+#pragma unroll
+      for (int o = 1; o < 8; o <<= 1) {
+        vu += __shfl_xor_sync(0xffffffffu, vu, o);
+        if (ACT == ACT_SWIGLU) vg += __shfl_xor_sync(0xffffffffu, vg, o);
+      }
+      // lanes 8g hold neuron g's sums: membership and activation there, then broadcast
+      float a_l = 0.f;
+      const int g_l = lane >> 3;
+      if ((lane & 7) == 0 && g_l < ng) {
+        const int i = S.meta[s].ids[g_l];
+        const int m = (i - c) / G;
+        const int kl = m / kTN;
+        if ((S.own_bits[kl] >> (m % kTN)) & 1u) {
+          if (ACT == ACT_RELU)
+            a_l = fmaxf(vu + S.own_bup[kl][m % kTN], 0.f);
+          else
+            a_l = silu(vg) * vu;
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < kMaxGN; ++g) av[g] = __shfl_sync(0xffffffffu, a_l, 8 * g);
+    }
+    // down-projection rows: y += a_g * W2T_g (every thread, its own chunks)
 #pragma unroll
     for (int g = 0; g < kMaxGN; ++g) {
-      if (g < ng) {
-        float up = 0.f, gt = 0.f;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) {
-          up += S.red[par][w][2 * g];
-          gt += S.red[par][w][2 * g + 1];
-        }
-        const int i = S.meta[s].ids[g];
-        const int tile = i / kTN;
-        const bool member = (S.own_bits[(tile - c) / G] >> (i % kTN)) & 1u;
-        float av;
-        if (ACT == ACT_RELU)
-          av = member ? fmaxf(up + __ldg(a.b_up + i), 0.f) : 0.f;
-        else
-          av = member ? silu(gt) * up : 0.f;
-        if (av != 0.f) {
-          const uint8_t *nd = S.ring[s] + g * NL.bytes;
+      for (int cq = 0; cq < CPT; ++cq) {
+        if (WT == W_F16) {
+          float w[8];
+          h8_to_f8(*reinterpret_cast<const uint4 *>(nd[g] + NL.down + coff[cq] * 16), w);
 #pragma unroll
-          for (int cq = 0; cq < CPT; ++cq) {
-            const int ch = tid + cq * kConsumers;
-            if (ch < nch) {
-              if (WT == W_F16) {
-                float w[8];
-                h8_to_f8(*reinterpret_cast<const uint4 *>(nd + NL.down + ch * 16), w);
+          for (int e = 0; e < 8; ++e) y[cq][e] = fmaf(av[g], w[e], y[cq][e]);
+        } else {
+          const float sd = __half2float(*reinterpret_cast<const __half *>(nd[g] + NL.sdown + (coff[cq] >> 1) * 2));
+          const uint2 wq = *reinterpret_cast<const uint2 *>(nd[g] + NL.down + coff[cq] * 8);
+          const float as = av[g] * sd;
+          uint32_t qh[8];
+          q8_to_h2(wq.x, qh);
+          q8_to_h2(wq.y, qh + 4);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) y[cq][e] = fmaf(av, w[e], y[cq][e]);
-              } else {
-                const float sd = __half2float(*reinterpret_cast<const __half *>(nd + NL.sdown + (ch >> 1) * 2));
-                const uint2 wq = *reinterpret_cast<const uint2 *>(nd + NL.down + ch * 8);
-                const uint32_t ws[2] = {wq.x, wq.y};
-                const float as = av * sd;
-#pragma unroll
-                for (int j = 0; j < 2; ++j)
-#pragma unroll
-                  for (int e = 0; e < 8; ++e)
-                    y[cq][8 * j + e] = fmaf(as, (float)((int)((ws[j] >> (4 * e)) & 15u) - 8), y[cq][8 * j + e]);
-              }
-            }
+          for (int k = 0; k < 8; ++k) {
+            const float2 v = __half22float2(*reinterpret_cast<const __half2 *>(&qh[k]));
+            y[cq][2 * k] = fmaf(as, v.x, y[cq][2 * k]);
+            y[cq][2 * k + 1] = fmaf(as, v.y, y[cq][2 * k + 1]);
           }
         }
       }
@@ -681,8 +818,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Args a) {
   for (int base = c0; base < c1; base += 32) {
     const int col = base + col_l;
     float sum = 0.f;
-    if (col < c1)
-      for (int cc = grp; cc < G; cc += kConsumerWarps) sum += ld_cg(a.partial + (size_t)cc * d + col);
+    if (col < c1) {
+      constexpr int kMaxPer = 40;  // G <= 320
+      float v[kMaxPer];
+#pragma unroll
+      for (int q = 0; q < kMaxPer; ++q) {
+        const int cc = grp + q * kConsumerWarps;
+        v[q] = (cc < G) ? ld_cg(a.partial + (size_t)cc * d + col) : 0.f;
+      }
+#pragma unroll
+      for (int q = 0; q < kMaxPer; ++q) sum += v[q];
+    }
     S.fin[grp][col_l] = sum;
     consumer_sync();
     if (grp == 0 && col < c1) {
@@ -694,40 +840,38 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Args a) {
     consumer_sync();
   }
 
-  // ---- ascending active ids (optional): CTA c writes the ids of tiles
-  // [c * tpc, (c + 1) * tpc) after the popcount of all earlier tiles
+  // ---- ascending active ids (optional): CTA c writes the ids of words
+  // [c * tpc, (c + 1) * tpc) after the popcount of all earlier words
   if (a.idx != nullptr || a.count != nullptr) {
-    const int tpc = (ntiles + G - 1) / G;
-    const int t0 = min(ntiles, c * tpc), t1 = min(ntiles, t0 + tpc);
-    int before = 0;
-    for (int t = tid; t < t0; t += kConsumers) before += __popc((unsigned)__ldcg(a.mask16 + t));
-    int total = before;
-    for (int t = t0 + tid; t < ntiles; t += kConsumers) total += __popc((unsigned)__ldcg(a.mask16 + t));
+    const int tpc = (nwords + G - 1) / G;
+    const int t0 = min(nwords, c * tpc), t1 = min(nwords, t0 + tpc);
+    int before = 0, total = 0;
+    for (int t = tid; t < nwords; t += kConsumers) {
+      const int pc = __popc(__ldcg(a.mask32 + t));
+      total += pc;
+      if (t < t0) before += pc;
+    }
     before = __reduce_add_sync(0xffffffffu, before);
     total = __reduce_add_sync(0xffffffffu, total);
-    if (lane == 0) S.iscan[warp] = before;
-    consumer_sync();
-    if (tid == 0) {
-      int b = 0;
-      for (int w = 0; w < kConsumerWarps; ++w) b += S.iscan[w];
-      S.iscan[0] = b;
+    if (lane == 0) {
+      S.iscan[warp] = before;
+      S.dred[warp] = (double)total;
     }
     consumer_sync();
-    before = S.iscan[0];
-    consumer_sync();
-    if (lane == 0) S.iscan[warp] = total;
-    consumer_sync();
     if (tid == 0) {
-      int tt = 0;
-      for (int w = 0; w < kConsumerWarps; ++w) tt += S.iscan[w];
+      int b = 0, tt = 0;
+      for (int w = 0; w < kConsumerWarps; ++w) {
+        b += S.iscan[w];
+        tt += (int)S.dred[w];
+      }
       if (c == 0 && a.count) a.count[0] = tt;
       if (a.idx) {
-        int pos = before;
+        int pos = b;
         for (int t = t0; t < t1; ++t) {
-          unsigned b = (unsigned)__ldcg(a.mask16 + t);
-          while (b) {
-            const int bit = __ffs(b) - 1;
-            b &= b - 1u;
+          unsigned bits = __ldcg(a.mask32 + t);
+          while (bits) {
+            const int bit = __ffs(bits) - 1;
+            bits &= bits - 1u;
             a.idx[pos++] = t * kTN + bit;
           }
         }

@@ -9,9 +9,9 @@ f = 16384, rank-1024 predictor, mean firing rate 10%, hot prefix 20%) at
 batch 1.  Steps rotate through 8 independently seeded layer replicas (2.5 GB,
 far above the 126 MB L2) and 32 seeded tokens, so weights come from HBM.
 
-Metric: achieved HBM GB/s over the bytes the step must touch (predictor
-weights + up rows of the predicted union + down rows of the neurons with a
-nonzero activation + token in / y out), with us per layer alongside.  Timed
+Metric: achieved HBM GB/s over the bytes the step touches (predictor weights
+and bias + up/gate and down rows of the predicted union + token in / y out),
+with us per layer alongside.  Timed
 with CUDA events around graph replays; N > 1 GPUs run independent replicas
 (weak scaling, no collective on the data path) and the time is the maximum
 over ranks.
@@ -130,14 +130,14 @@ def predictor_bytes(cfg: inputs.Config) -> int:
     return (cfg.r * cfg.d + cfg.f * cfg.r) * e + 4 * cfg.f
 
 
-def step_bytes(cfg: inputs.Config, B: int, n_up_rows: int, n_live: int) -> int:
-    """Bytes one step must move: predictor, up (and gate) rows of the union
-    (plus bias), down rows of the neurons with a nonzero value, u in, y out."""
-    n_mat_up = 2 if cfg.act == "swiglu" else 1
+def step_bytes(cfg: inputs.Config, B: int, n_union: int) -> int:
+    """Bytes of one step: predictor factors and bias, the up (and gate) and
+    down rows of the union of the predicted sets (plus the ReLU bias), u in and
+    y out."""
+    n_mat = 3 if cfg.act == "swiglu" else 2
     ue = 4 if cfg.wtype == "f32" else 2
     bias = 4 if cfg.act == "relu" else 0
-    return (predictor_bytes(cfg) + n_up_rows * (n_mat_up * row_bytes(cfg) + bias) + n_live * row_bytes(cfg)
-            + B * cfg.d * ue + B * cfg.d * 4)
+    return (predictor_bytes(cfg) + n_union * (n_mat * row_bytes(cfg) + bias) + B * cfg.d * ue + B * cfg.d * 4)
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -210,13 +210,8 @@ def oracle_run(layer_host: inputs.LayerTensors, cfg, u_host: torch.Tensor, secon
         y = oracle.ffn_masked(L, u, pr["idx"])
         dt = time.perf_counter() - t0
         union = np.unique(np.concatenate(pr["idx"])) if len(pr["idx"]) else np.array([], np.int64)
-        if cfg.act == "relu":
-            phi = oracle.neuron_phi(L, u)  # untimed bookkeeping of the live rows
-            live = int(np.sum(np.any(phi[:, union] != 0, axis=0))) if len(union) else 0
-        else:
-            live = len(union)
         t_tot += dt
-        b_tot += step_bytes(cfg, u.shape[0], len(union), live)
+        b_tot += step_bytes(cfg, u.shape[0], len(union))
         n += 1
         if t_tot >= seconds:
             break
@@ -275,16 +270,7 @@ def bench_ours(args, world, rank, local):
             c = cnt.cpu().tolist()
             sets = [idx[b, :c[b]].long() for b in range(B)]
             union = torch.unique(torch.cat(sets)) if sum(c) else torch.empty(0, dtype=torch.long, device=dev)
-            if cfg.act == "relu" and len(union):
-                W = lt.w_up.index_select(0, union).float()
-                pre = toks[t].float() @ W.T + lt.b_up[union]
-                member = torch.zeros((B, len(union)), dtype=torch.bool, device=dev)
-                for b in range(B):
-                    member[b] = torch.isin(union, sets[b])
-                live = int(((pre > 0) & member).any(0).sum())
-            else:
-                live = len(union)
-            pair_bytes[(r, t)] = step_bytes(cfg, B, len(union), live)
+            pair_bytes[(r, t)] = step_bytes(cfg, B, len(union))
     assert pb.pi_get_device_status(ws) == 0
 
     # graphs: one of S = lcm(R, T) steps, plus single-step graphs for a remainder
