@@ -140,9 +140,10 @@ PI_DEV bool mbar_test(unsigned long long *b, unsigned parity) {
       : "memory");
   return ok != 0;
 }
-// bounded wait; false on timeout (status recorded)
-PI_DEV bool mbar_wait(unsigned long long *b, unsigned parity, int *status) {
-  if (mbar_test(b, parity)) return true;
+// bounded wait; false on timeout (status recorded).  The fast path (phase
+// already complete) is inline, the suspending loop is out of line to keep
+// the consumer loop small in the instruction cache.
+__device__ __noinline__ bool mbar_wait_slow(unsigned long long *b, unsigned parity, int *status) {
   const unsigned long long t0 = globaltimer();
   for (;;) {
     if (mbar_try(b, parity, 20000u)) return true;
@@ -151,6 +152,10 @@ PI_DEV bool mbar_wait(unsigned long long *b, unsigned parity, int *status) {
       return false;
     }
   }
+}
+PI_DEV bool mbar_wait(unsigned long long *b, unsigned parity, int *status) {
+  if (mbar_test(b, parity)) return true;
+  return mbar_wait_slow(b, parity, status);
 }
 PI_DEV void bulk_g2s(void *dst, const void *src, unsigned bytes, unsigned long long *bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
@@ -307,8 +312,12 @@ struct NeuronLayout {
 PI_DEV int own_count(int f, int c, int G) { return c < f ? (f - 1 - c) / G + 1 : 0; }
 
 // ---------------------------------------------------------------- producer
+// The whole producer warp runs this loop in lockstep with identical state;
+// lane 0 writes the slot descriptors and arms the mbarriers, and the bulk
+// copies of an item are spread over the lanes (one row per lane), so a tile
+// of 32 strided rows costs one warp instruction.
 template <int WT, int ACT>
-PI_DEV void producer(Smem &S, const Args &a, int c, int G) {
+PI_DEV void producer(Smem &S, const Args &a, int c, int G, int lane) {
   const int d = a.d, f = a.f, r = a.r;
   const int nn = own_count(f, c, G);
   const int nown = (nn + kTN - 1) / kTN;
@@ -317,26 +326,44 @@ PI_DEV void producer(Smem &S, const Args &a, int c, int G) {
   const NeuronLayout<WT, ACT> NL(d);
   const int GN = min(kMaxGN, kSlotBytes / (int)NL.bytes);
   const unsigned rb = wrow_bytes<WT>(d), sb = srow_bytes<WT>(d);
+  constexpr int CPN = (ACT == ACT_SWIGLU ? 3 : 2) * (WT == W_INT4 ? 2 : 1);  // copies per neuron
   const bool want_mask = a.idx != nullptr || a.count != nullptr;
-  unsigned pn = 0;       // items issued
-  int k = 0;             // own tiles issued
-  int hk = 0;            // own tiles harvested
-  int act_tail = 0;      // fired ids appended (index mode)
-  int taken = 0;         // fired ids issued as gather items
+  unsigned pn = 0;   // items issued
+  int k = 0;         // own tiles issued
+  int hk = 0;        // own tiles harvested
+  int act_tail = 0;  // fired own indices appended (index mode)
+  int taken = 0;     // fired own indices issued as gather items
   bool ok = true;
 
   // fired bits of own tile hk are final once its slot's empty phase completed
   auto harvest = [&]() {
     const int s = S.tile_item[hk] % kSlots;
-    unsigned b = S.tbits[s];
+    const unsigned bits = S.tbits[s];
+    const int fired = __popc(bits);
+    if (lane == 0) {
+      unsigned b = bits;
+      int t = act_tail;
+      while (b) {
+        const int q = __ffs(b) - 1;
+        b &= b - 1u;
+        const int m = hk * kTN + q;
+        const int i = c + m * G;
+        if (want_mask) atomicOr(a.mask32 + (i >> 5), 1u << (i & 31));
+        if (i >= a.H) S.act[t++] = m;
+      }
+    }
+    // prefix neurons were issued densely: count only the others (ids grow with q)
+    int added = 0;
+    unsigned b = bits;
     while (b) {
       const int q = __ffs(b) - 1;
       b &= b - 1u;
-      const int i = c + (hk * kTN + q) * G;
-      if (want_mask) atomicOr(a.mask32 + (i >> 5), 1u << (i & 31));
-      if (i >= a.H) S.act[act_tail++] = i;
+      added += (c + (hk * kTN + q) * G >= a.H) ? 1 : 0;
     }
+    (void)fired;
+    act_tail += added;
     ++hk;
+    __syncwarp();
   };
   auto tile_done = [&](int kk) -> bool {
     const unsigned it = (unsigned)S.tile_item[kk];
@@ -348,33 +375,55 @@ PI_DEV void producer(Smem &S, const Args &a, int c, int G) {
     s = (int)(pn % kSlots);
     const unsigned par = ((pn / kSlots) & 1u) ^ 1u;
     if (!mbar_wait(&S.empty[s], par, a.status)) {
-      S.abort_flag = 1;
+      if (lane == 0) S.abort_flag = 1;
       return false;
     }
     while (hk < k && (unsigned)S.tile_item[hk] + kSlots <= pn) harvest();
     return true;
   };
-  auto issue_gather = [&](const int *ids, int n) -> bool {
+  // gather item: own indices ms[0..n); lane j issues copy j
+  auto issue_gather = [&](const int *ms, int n) -> bool {
     int s;
     if (!acquire(s)) return false;
-    SlotMeta &m = S.meta[s];
-    m.type = IT_GATHER;
-    m.n = n;
-    m.first = 0;
-    for (int g = 0; g < n; ++g) m.ids[g] = ids[g];
-    mbar_arrive_tx(&S.full[s], NL.bytes * (unsigned)n);
-    uint8_t *dst = S.ring[s];
-    for (int g = 0; g < n; ++g) {
-      const size_t i = (size_t)ids[g];
-      uint8_t *nd = dst + g * NL.bytes;
-      bulk_g2s(nd + NL.up, (const char *)a.w_up + i * rb, rb, &S.full[s]);
-      if (ACT == ACT_SWIGLU) bulk_g2s(nd + NL.gate, (const char *)a.w_gate + i * rb, rb, &S.full[s]);
-      bulk_g2s(nd + NL.down, (const char *)a.w_down_t + i * rb, rb, &S.full[s]);
-      if (WT == W_INT4) {
-        bulk_g2s(nd + NL.sup, (const char *)a.s_up + i * sb, sb, &S.full[s]);
-        if (ACT == ACT_SWIGLU) bulk_g2s(nd + NL.sgate, (const char *)a.s_gate + i * sb, sb, &S.full[s]);
-        bulk_g2s(nd + NL.sdown, (const char *)a.s_down_t + i * sb, sb, &S.full[s]);
+    if (lane == 0) {
+      SlotMeta &m = S.meta[s];
+      m.type = IT_GATHER;
+      m.n = n;
+      m.first = 0;
+      for (int g = 0; g < n; ++g) m.ids[g] = ms[g];
+      mbar_arrive_tx(&S.full[s], NL.bytes * (unsigned)n);
+    }
+    __syncwarp();
+    if (lane < n * CPN) {
+      const int g = lane / CPN, kind = lane % CPN;
+      const size_t i = (size_t)(c + ms[g] * G);
+      uint8_t *nd = S.ring[s] + g * NL.bytes;
+      const void *src;
+      unsigned off, bytes = rb;
+      if (kind == 0) {
+        src = (const char *)a.w_up + i * rb;
+        off = NL.up;
+      } else if (ACT == ACT_SWIGLU && kind == 1) {
+        src = (const char *)a.w_gate + i * rb;
+        off = NL.gate;
+      } else if (kind == (ACT == ACT_SWIGLU ? 2 : 1)) {
+        src = (const char *)a.w_down_t + i * rb;
+        off = NL.down;
+      } else {  // int4 scale rows, in the order up, [gate,] down
+        const int sk = kind - (ACT == ACT_SWIGLU ? 3 : 2);
+        bytes = sb;
+        if (sk == 0) {
+          src = (const char *)a.s_up + i * sb;
+          off = NL.sup;
+        } else if (ACT == ACT_SWIGLU && sk == 1) {
+          src = (const char *)a.s_gate + i * sb;
+          off = NL.sgate;
+        } else {
+          src = (const char *)a.s_down_t + i * sb;
+          off = NL.sdown;
+        }
       }
+      bulk_g2s(nd + off, src, bytes, &S.full[s]);
     }
     ++pn;
     return true;
@@ -385,12 +434,14 @@ PI_DEV void producer(Smem &S, const Args &a, int c, int G) {
     const int n = min(rpi, j1 - j);
     int s;
     if (!(ok = acquire(s))) break;
-    S.meta[s].type = IT_P1;
-    S.meta[s].n = n;
-    S.meta[s].first = j;
-    const unsigned bytes = (unsigned)n * (unsigned)d * 2u;
-    mbar_arrive_tx(&S.full[s], bytes);
-    bulk_g2s(S.ring[s], a.p1 + (size_t)j * d, bytes, &S.full[s]);
+    if (lane == 0) {
+      S.meta[s].type = IT_P1;
+      S.meta[s].n = n;
+      S.meta[s].first = j;
+      const unsigned bytes = (unsigned)n * (unsigned)d * 2u;
+      mbar_arrive_tx(&S.full[s], bytes);
+      bulk_g2s(S.ring[s], a.p1 + (size_t)j * d, bytes, &S.full[s]);
+    }
     ++pn;
   }
   // 2. predictor tiles and gather rows
@@ -406,28 +457,29 @@ PI_DEV void producer(Smem &S, const Args &a, int c, int G) {
       const int rows = min(kTN, nn - k * kTN);
       int s;
       if (!(ok = acquire(s))) break;
-      S.meta[s].type = IT_P2;
-      S.meta[s].n = rows;
-      S.meta[s].first = k;
-      S.tbits[s] = 0u;
-      S.tile_item[k] = (int)pn;
       const unsigned rbp = (unsigned)r * 2u;
-      mbar_arrive_tx(&S.full[s], (unsigned)rows * rbp);
-      for (int q = 0; q < rows; ++q)
-        bulk_g2s(S.ring[s] + q * rbp, a.p2 + (size_t)(c + (k * kTN + q) * G) * r, rbp, &S.full[s]);
+      if (lane == 0) {
+        S.meta[s].type = IT_P2;
+        S.meta[s].n = rows;
+        S.meta[s].first = k;
+        S.tbits[s] = 0u;
+        S.tile_item[k] = (int)pn;
+        mbar_arrive_tx(&S.full[s], (unsigned)rows * rbp);
+      }
+      __syncwarp();
+      if (lane < rows) bulk_g2s(S.ring[s] + lane * rbp, a.p2 + (size_t)(c + (k * kTN + lane) * G) * r, rbp, &S.full[s]);
       ++pn;
       // dense hot prefix: the tile's prefix neurons (the smallest ids), now
-      int ids[kMaxGN], ng = 0;
+      int ms[kMaxGN], ng = 0;
       for (int q = 0; ok && q < rows; ++q) {
-        const int i = c + (k * kTN + q) * G;
-        if (i >= a.H) break;
-        ids[ng++] = i;
+        if (c + (k * kTN + q) * G >= a.H) break;
+        ms[ng++] = k * kTN + q;
         if (ng == GN) {
-          ok = issue_gather(ids, ng);
+          ok = issue_gather(ms, ng);
           ng = 0;
         }
       }
-      if (ok && ng) ok = issue_gather(ids, ng);
+      if (ok && ng) ok = issue_gather(ms, ng);
       ++k;
       continue;
     }
@@ -435,7 +487,7 @@ PI_DEV void producer(Smem &S, const Args &a, int c, int G) {
     // wait for the consumers to finish the oldest unharvested tile
     const unsigned it = (unsigned)S.tile_item[hk];
     if (!mbar_wait(&S.empty[it % kSlots], (it / kSlots) & 1u, a.status)) {
-      S.abort_flag = 1;
+      if (lane == 0) S.abort_flag = 1;
       ok = false;
       break;
     }
@@ -445,10 +497,12 @@ PI_DEV void producer(Smem &S, const Args &a, int c, int G) {
   __threadfence();  // mask words visible before the consumers' grid barrier
   int s;
   if (acquire(s)) {
-    S.meta[s].type = IT_DONE;
-    S.meta[s].n = 0;
-    mbar_arrive(&S.full[s]);
-  } else {
+    if (lane == 0) {
+      S.meta[s].type = IT_DONE;
+      S.meta[s].n = 0;
+      mbar_arrive(&S.full[s]);
+    }
+  } else if (lane == 0) {
     S.abort_flag = 1;
   }
 }
@@ -480,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Args a) {
   __syncthreads();
 
   if (warp == kConsumerWarps) {
-    if (lane == 0) producer<WT, ACT>(S, a, c, G);
+    producer<WT, ACT>(S, a, c, G, lane);
     return;
   }
 
@@ -644,7 +698,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Args a) {
       const int kl = S.meta[s].first, rows = S.meta[s].n;
       constexpr int RPW = kTN / kConsumerWarps;
       unsigned b = 0u;
-#pragma unroll
+#pragma unroll 1
       for (int rp = 0; rp < RPW; rp += 2) {
         uint4 wv[2][4];
 #pragma unroll
@@ -733,7 +787,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Args a) {
     // sum the 8 warps' partials: lane (g, w) = (lane / 8, lane % 8) loads
     // warp w's partial of neuron g, a 3-step butterfly over the 8 lanes of a
     // group adds them in a fixed order, and shuffles broadcast the sums
-    float av[kMaxGN];
+    float a_l = 0.f;  // on lanes 8g: value of neuron g
     {
       static_assert(kMaxGN * kConsumerWarps == 32, "one lane per (neuron, warp)");
       float vu = S.red[par][lane & 7][2 * (lane >> 3)];
@@ -743,12 +797,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Args a) {
         vu += __shfl_xor_sync(0xffffffffu, vu, o);
         if (ACT == ACT_SWIGLU) vg += __shfl_xor_sync(0xffffffffu, vg, o);
       }
-      // lanes 8g hold neuron g's sums: membership and activation there, then broadcast
-      float a_l = 0.f;
+      // lanes 8g hold neuron g's sums: membership and activation there
       const int g_l = lane >> 3;
       if ((lane & 7) == 0 && g_l < ng) {
-        const int i = S.meta[s].ids[g_l];
-        const int m = (i - c) / G;
+        const int m = S.meta[s].ids[g_l];  // own index: neuron c + m G
         const int kl = m / kTN;
         if ((S.own_bits[kl] >> (m % kTN)) & 1u) {
           if (ACT == ACT_RELU)
@@ -757,31 +809,33 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Args a) {
             a_l = silu(vg) * vu;
         }
       }
-#pragma unroll
-      for (int g = 0; g < kMaxGN; ++g) av[g] = __shfl_sync(0xffffffffu, a_l, 8 * g);
     }
-    // down-projection rows: y += a_g * W2T_g (every thread, its own chunks)
-#pragma unroll
-    for (int g = 0; g < kMaxGN; ++g) {
+    // down-projection rows: y += a_g * W2T_g (every thread, its own chunks);
+    // a_g is the same in every thread, so skipping zeros never diverges
+#pragma unroll 1
+    for (int g = 0; g < ng; ++g) {
+      const float ag = __shfl_sync(0xffffffffu, a_l, 8 * g);
+      if (ag == 0.f) continue;
+      const uint8_t *ndg = S.ring[s] + g * NL.bytes;
 #pragma unroll
       for (int cq = 0; cq < CPT; ++cq) {
         if (WT == W_F16) {
           float w[8];
-          h8_to_f8(*reinterpret_cast<const uint4 *>(nd[g] + NL.down + coff[cq] * 16), w);
+          h8_to_f8(*reinterpret_cast<const uint4 *>(ndg + NL.down + coff[cq] * 16), w);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) y[cq][e] = fmaf(av[g], w[e], y[cq][e]);
+          for (int e = 0; e < 8; ++e) y[cq][e] = fmaf(ag, w[e], y[cq][e]);
         } else {
-          const float sd = __half2float(*reinterpret_cast<const __half *>(nd[g] + NL.sdown + (coff[cq] >> 1) * 2));
-          const uint2 wq = *reinterpret_cast<const uint2 *>(nd[g] + NL.down + coff[cq] * 8);
-          const float as = av[g] * sd;
+          const float sd = __half2float(*reinterpret_cast<const __half *>(ndg + NL.sdown + (coff[cq] >> 1) * 2));
+          const uint2 wq = *reinterpret_cast<const uint2 *>(ndg + NL.down + coff[cq] * 8);
+          const float as = ag * sd;
           uint32_t qh[8];
           q8_to_h2(wq.x, qh);
           q8_to_h2(wq.y, qh + 4);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const float2 v = __half22float2(*reinterpret_cast<const __half2 *>(&qh[k]));
-            y[cq][2 * k] = fmaf(as, v.x, y[cq][2 * k]);
-            y[cq][2 * k + 1] = fmaf(as, v.y, y[cq][2 * k + 1]);
+          for (int kq = 0; kq < 8; ++kq) {
+            const float2 v = __half22float2(*reinterpret_cast<const __half2 *>(&qh[kq]));
+            y[cq][2 * kq] = fmaf(as, v.x, y[cq][2 * kq]);
+            y[cq][2 * kq + 1] = fmaf(as, v.y, y[cq][2 * kq + 1]);
           }
         }
       }

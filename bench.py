@@ -140,6 +140,40 @@ def step_bytes(cfg: inputs.Config, B: int, n_union: int) -> int:
     return (predictor_bytes(cfg) + n_union * (n_mat * row_bytes(cfg) + bias) + B * cfg.d * ue + B * cfg.d * 4)
 
 
+# ----------------------------------------------------------------------------- profile summaries
+
+def kernel_source_hash() -> str:
+    """Hash of the CUDA sources; a profile summary's counters apply only to the
+    kernels built from the sources it records."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "activation_sparse_decode_gemv_b200", "csrc", "*"))):
+        with open(p, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(summary: str):
+    """DRAM bytes per launch (read + write) from a profiles/ summary, or None
+    when the summary is missing or was taken on other kernel sources."""
+    path = os.path.join(ROOT, "profiles", summary)
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    with open(path) as fh:
+        for line in fh:
+            if ":" in line and line.startswith("- "):
+                k, v = line[2:].split(":", 1)
+                fields[k.strip()] = v.strip().strip("`")
+    if fields.get("source_hash") != kernel_source_hash():
+        return None
+    try:
+        return float(fields["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -367,7 +401,9 @@ def bench_ours(args, world, rank, local):
                    "l2": f"{R} rotating seeded replicas ({sum(l.nbytes() for l in layers) / 1e9:.1f} GB) > L2",
                    "bytes_per_step": nbytes / args.steps, "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm", "achieved": per_gpu, "peak": peak, "unit": "GB/s", "frac": per_gpu / peak,
-                     "traffic": None,
+                     "traffic": (profiled_traffic(f"decode_fused_kernel_{cfg.name}_batch{B}.md")
+                                 if kernels_per_step(cfg, B) == 1 else None),
+                     "algorithmic_bytes_per_launch": nbytes / args.steps,
                      "kernel": ("decode_fused_kernel (the whole step is one launch)" if kernels_per_step(cfg, B) == 1
                                 else "whole decode step (5 kernels)"),
                      "peak_source": "measured" if "hbm_gbs" in peaks else "fallback"},
