@@ -22,13 +22,15 @@ PI_ERR_CUDA, PI_ERR_TIMEOUT, PI_ERR_DEVICE_STATUS, PI_ERR_WORKSPACE = 4, 5, 6, 7
 PI_ACT_RELU, PI_ACT_SWIGLU = 0, 1
 PI_W_F32, PI_W_F16, PI_W_INT4G32 = 0, 1, 2
 PI_FFN_ACCUMULATE, PI_FFN_HOT_DENSE, PI_FFN_HOT_INDEX = 1, 2, 4
+PI_STATIC_SCRATCH_BYTES = 4 * 1024 * 1024  # device scratch of pi_decode_ffn_static
 
 WTYPE = {"f32": PI_W_F32, "f16": PI_W_F16, "int4g32": PI_W_INT4G32}
 ACT = {"relu": PI_ACT_RELU, "swiglu": PI_ACT_SWIGLU}
 
 # every symbol the header declares
 EXPORTS = ("pi_ffn_create", "pi_ffn_destroy", "pi_workspace_size", "pi_workspace_init", "pi_predict",
-           "pi_sparse_ffn", "pi_decode_ffn", "pi_decode_ffn_stack", "pi_get_device_status", "pi_status_string")
+           "pi_sparse_ffn", "pi_decode_ffn", "pi_decode_ffn_stack", "pi_decode_ffn_static", "pi_get_device_status",
+           "pi_status_string")
 
 
 class PiError(RuntimeError):
@@ -66,11 +68,12 @@ def lib() -> C.CDLL:
         L.pi_sparse_ffn.argtypes = [vp, vp, i, vp, vp, vp, C.c_uint, vp, sz, vp]
         L.pi_decode_ffn.argtypes = [vp, vp, i, vp, vp, vp, C.c_uint, vp, sz, vp]
         L.pi_decode_ffn_stack.argtypes = [C.POINTER(vp), i, vp, i, vp, vp, C.c_uint, vp, sz, vp]
+        L.pi_decode_ffn_static.argtypes = [vp, vp, vp, vp, vp, C.c_uint, vp, vp]
         L.pi_get_device_status.argtypes = [vp, vp, C.POINTER(i)]
         L.pi_status_string.argtypes = [i]
         L.pi_status_string.restype = C.c_char_p
         for n in ("pi_ffn_create", "pi_workspace_size", "pi_workspace_init", "pi_predict", "pi_sparse_ffn",
-                  "pi_decode_ffn", "pi_decode_ffn_stack", "pi_get_device_status"):
+                  "pi_decode_ffn", "pi_decode_ffn_stack", "pi_decode_ffn_static", "pi_get_device_status"):
             getattr(L, n).restype = C.c_int
         _lib = L
     return _lib
@@ -171,6 +174,15 @@ def pi_decode_ffn(layer: FfnLayer, u: torch.Tensor, y: torch.Tensor, ws: torch.T
     B = u.shape[0]
     _check(lib().pi_decode_ffn(layer.handle, _p(u), B, _p(y), _p(idx), _p(count), int(flags), *_wsargs(ws),
                                _stream(stream)), "pi_decode_ffn")
+
+
+def pi_decode_ffn_static(layer: FfnLayer, u: torch.Tensor, y: torch.Tensor, idx: Optional[torch.Tensor] = None,
+                         count: Optional[torch.Tensor] = None, flags: int = 0,
+                         dev_status: Optional[torch.Tensor] = None, stream=None):
+    """Batch-1 decode step on the library's static device scratch (no workspace)."""
+    assert u.numel() == layer.d and y.numel() == layer.d, "pi_decode_ffn_static is batch 1"
+    _check(lib().pi_decode_ffn_static(layer.handle, _p(u), _p(y), _p(idx), _p(count), int(flags), _p(dev_status),
+                                      _stream(stream)), "pi_decode_ffn_static")
 
 
 def pi_decode_ffn_stack(layers: Sequence[FfnLayer], x: torch.Tensor, ws: torch.Tensor,

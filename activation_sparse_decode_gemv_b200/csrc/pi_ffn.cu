@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 #include <new>
 
 #include "pi_ffn.h"
@@ -395,6 +396,38 @@ pi_status check_call(const pi_ffn *h, int B) {
 
 }  // namespace
 
+// ---------------------------------------------------------------- static scratch
+// Device scratch for pi_decode_ffn_static, for callers that cannot allocate
+// device memory at decode time (no allocator handle of their own, HBM fully
+// reserved by their caching allocator, or no tolerance for cudaMalloc's
+// implicit device synchronisation).  One array per device, loaded with the
+// module; it is laid out like a batch-1 workspace.
+static __device__ __align__(256) unsigned char g_static_scratch[PI_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxStaticDevices = 64;
+std::mutex g_static_mu;
+void *g_static_ptr[kMaxStaticDevices];
+
+// Device address of the scratch array on the current device, looked up once
+// per device (with that device current) and cached.
+pi_status static_scratch(void **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PI_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxStaticDevices) return PI_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (!g_static_ptr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return PI_ERR_CUDA;
+    g_static_ptr[dev] = p;
+  }
+  *out = g_static_ptr[dev];
+  return PI_OK;
+}
+
+}  // namespace
+
 // ====================================================================== API
 
 extern "C" {
@@ -534,6 +567,38 @@ pi_status pi_decode_ffn_stack(const pi_ffn_t *layers, int L, float *x, int B, in
     if ((s = run_predict(layers[l], w.u(), B, idx, fmax, cnt, w, st)) != PI_OK) return s;
     if ((s = run_ffn(layers[l], w.u(), B, x, 1, flags, w, st)) != PI_OK) return s;
   }
+  return PI_OK;
+}
+
+pi_status pi_decode_ffn_static(pi_ffn_t h, const void *u, float *y, int32_t *idx, int32_t *count, unsigned flags,
+                               int *dev_status, pi_stream_t stream) {
+  pi_status s = check_call(h, 1);
+  if (s != PI_OK) return s;
+  if (!u || !y) return PI_ERR_INVALID_ARG;
+  if (!aligned16(u) || !aligned16(y) || (idx && !aligned16(idx)) || (count && !aligned16(count)) ||
+      (reinterpret_cast<uintptr_t>(dev_status) & 3u))
+    return PI_ERR_MISALIGNED;
+  if (flags & ~7u) return PI_ERR_INVALID_ARG;
+  void *base = nullptr;
+  if ((s = static_scratch(&base)) != PI_OK) return s;
+  const int G = device_sm_count();
+  if (G <= 0) return PI_ERR_CUDA;
+  Ws w;
+  w.L = ws_layout(h->d.d_model, h->d.d_ffn, h->d.rank, 1, G);
+  w.base = static_cast<char *>(base);
+  if (w.L.total > PI_STATIC_SCRATCH_BYTES) return PI_ERR_WORKSPACE;
+  cudaStream_t st = (cudaStream_t)stream;
+  // status word, union count and grid-barrier word must start at zero; the
+  // kernels initialise the rest of the scratch they read
+  PI_CUDA(cudaMemsetAsync(base, 0, 16, st));
+  const int acc = (flags & PI_FFN_ACCUMULATE) ? 1 : 0;
+  if (fused_ok(h, 1, G)) {
+    s = run_fused(h, u, y, 0, acc, idx, count, flags, w, st);
+  } else if ((s = run_predict(h, u, 1, idx, h->d.d_ffn, count, w, st)) == PI_OK) {
+    s = run_ffn(h, u, 1, y, acc, flags, w, st);
+  }
+  if (s != PI_OK) return s;
+  if (dev_status) PI_CUDA(cudaMemcpyAsync(dev_status, base, sizeof(int), cudaMemcpyDeviceToDevice, st));
   return PI_OK;
 }
 

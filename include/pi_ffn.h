@@ -22,14 +22,16 @@
  *    the duration of the call (or of the stream work it enqueues).  The
  *    library never allocates device memory; the caller allocates the
  *    workspace (size from pi_workspace_size) and every input and output.
+ *    The one exception to the workspace rule is pi_decode_ffn_static, which
+ *    uses a fixed-size device array of the library instead.
  *  - Row-major layouts.  fp16 is IEEE binary16.  int4g32: each neuron row is
  *    d/2 bytes of packed nibbles (element 2k in the low nibble of byte k,
  *    2k+1 in the high nibble) with one fp16 scale per 32 consecutive elements
  *    in a separate [f x d/32] array; value = scale * (q - 8).
  *  - Work is enqueued on the given stream (a cudaStream_t; NULL = legacy
  *    default stream) and is asynchronous; nothing synchronises the host
- *    except pi_get_device_status.  No call allocates, so all of them may be
- *    captured into a CUDA graph.
+ *    except pi_get_device_status.  No call allocates; the entry points that
+ *    take a workspace may be captured into a CUDA graph.
  *  - Argument errors are detected on the host before anything is launched
  *    and returned synchronously; nothing is enqueued then.  Problems only the
  *    device can see (an out-of-range id in a caller's list, a bounded wait
@@ -144,6 +146,42 @@ pi_status pi_decode_ffn(pi_ffn_t h, const void *u, int B, float *y, int32_t *idx
  * (l*B + b)*f_max), count_trace: optional [L x B]. */
 pi_status pi_decode_ffn_stack(const pi_ffn_t *layers, int L, float *x, int B, int32_t *idx_trace,
                               int32_t *count_trace, unsigned flags, void *ws, size_t ws_bytes, pi_stream_t stream);
+
+/* Size in bytes of the library's file-scope device scratch array, the only
+ * device memory pi_decode_ffn_static uses besides its arguments. */
+#define PI_STATIC_SCRATCH_BYTES (4u * 1024u * 1024u)
+
+/* pi_decode_ffn at batch 1 without a caller workspace and without allocating.
+ * The pages have no counterpart: this is an integration entry point only.
+ *
+ * Who needs it: callers that cannot call cudaMalloc (or own no device
+ * allocator) at decode time -- a plugin inside a runtime that hands out no
+ * device memory, an engine whose caching allocator has reserved all of HBM
+ * for weights and KV cache, or a latency-critical loop where cudaMalloc may
+ * synchronise the device.  Instead of a workspace, the call uses a
+ * PI_STATIC_SCRATCH_BYTES file-scope __device__ array of this library.  It
+ * calls no cudaMalloc / cudaFree or allocating library routine.
+ *
+ * u: [d] (fp16, or fp32 for PI_W_F32 layers); y: [d] fp32; idx/count:
+ * optional [f] / [1] int32 outputs as in pi_predict; flags: PI_FFN_*.
+ * dev_status: optional device int (4-byte aligned); when non-NULL it receives,
+ * in stream order, this call's device-side status (PI_OK, PI_ERR_TIMEOUT, ...).
+ *
+ * Limits and behaviour:
+ *  - The layer's batch-1 scratch (status words, h, mask words, union lists
+ *    and one d-float partial row per SM) must fit PI_STATIC_SCRATCH_BYTES;
+ *    otherwise the call returns PI_ERR_WORKSPACE and launches nothing.  On a
+ *    148-SM B200 this admits d_model <= 6928 at d_ffn = 16384 and rank 1024
+ *    (an OPT-7B- or LLaMA-13B-shaped layer, not OPT-30B or LLaMA-70B).
+ *  - The first call on each device does the set-up (looks up the array's
+ *    device address with the device current), so make it before any stream
+ *    capture.  Each call clears the scratch status and barrier words on the
+ *    stream before its kernels.
+ *  - There is one scratch array per device: calls that overlap on the GPU
+ *    (other streams, other host threads) race on it and give wrong results.
+ *    Serialise them, e.g. on one stream. */
+pi_status pi_decode_ffn_static(pi_ffn_t h, const void *u, float *y, int32_t *idx, int32_t *count, unsigned flags,
+                               int *dev_status, pi_stream_t stream);
 
 /* Synchronise the stream, read and clear the workspace status word.  *code is
  * PI_OK or the first device-side error recorded since the last read. */
