@@ -12,6 +12,7 @@
 #include "pi_ffn.h"
 #include "pi_fused.cuh"
 #include "pi_kernels.cuh"
+#include "pi_tc.cuh"
 
 struct pi_ffn {
   pi_ffn_desc d;
@@ -64,9 +65,47 @@ WsLayout ws_layout(int dmax, int fmax, int rmax, int B, int G) {
   return L;
 }
 
+// Tensor-core path (batch 16..32) scratch: token images, stream-K partials
+// and per-tile counters.  It sits at the END of the caller's buffer so its
+// counters keep their place whatever batch earlier calls used (they must stay
+// zero between calls; the kernels restore them).
+struct TcLayout {
+  size_t uimg, himg_hi, himg_lo, aimg, part, ctr_p1, ctr_p2, ctr_up, ctr_down, total;
+};
+
+TcLayout tc_layout(int dmax, int fmax, int rmax, int G) {
+  TcLayout L{};
+  size_t o = 0;
+  const size_t step_img = (size_t)pi::tc::kStepImg;
+  L.uimg = o;
+  o = align_up(o + (size_t)((dmax + 127) / 128) * step_img, 256);
+  L.himg_hi = o;
+  o = align_up(o + (size_t)((rmax + 127) / 128) * step_img, 256);
+  L.himg_lo = o;
+  o = align_up(o + (size_t)((rmax + 127) / 128) * step_img, 256);
+  L.aimg = o;
+  o = align_up(o + (size_t)((fmax + 127) / 128) * step_img, 256);
+  L.part = o;
+  o = align_up(o + (size_t)G * 2 * pi::tc::kPartFloats * 4, 256);
+  L.ctr_p1 = o;
+  o = align_up(o + (size_t)((rmax + 127) / 128) * 4, 256);
+  L.ctr_p2 = o;
+  o = align_up(o + (size_t)((fmax + 127) / 128) * 4, 256);
+  L.ctr_up = o;
+  o = align_up(o + (size_t)((fmax + 127) / 128) * 4, 256);
+  L.ctr_down = o;
+  o = align_up(o + (size_t)((dmax + pi::tc::kDownTileD - 1) / pi::tc::kDownTileD) * 4, 256);
+  L.total = o;
+  return L;
+}
+
+constexpr int kTcMinBatch = 16;
+
 struct Ws {
   WsLayout L;
+  TcLayout T;
   char *base;
+  char *tc;  // start of the tensor-core region (null when the call does not use it)
   int *status() const { return reinterpret_cast<int *>(base); }
   int32_t *ucount() const { return reinterpret_cast<int32_t *>(base) + 1; }
   unsigned *grid_bar() const { return reinterpret_cast<unsigned *>(base) + 2; }
@@ -77,6 +116,15 @@ struct Ws {
   int32_t *uprefix() const { return reinterpret_cast<int32_t *>(base + L.uprefix); }
   int32_t *ulist() const { return reinterpret_cast<int32_t *>(base + L.ulist); }
   float *partial() const { return reinterpret_cast<float *>(base + L.partial); }
+  unsigned char *uimg() const { return reinterpret_cast<unsigned char *>(tc + T.uimg); }
+  unsigned char *himg_hi() const { return reinterpret_cast<unsigned char *>(tc + T.himg_hi); }
+  unsigned char *himg_lo() const { return reinterpret_cast<unsigned char *>(tc + T.himg_lo); }
+  unsigned char *aimg() const { return reinterpret_cast<unsigned char *>(tc + T.aimg); }
+  float *tc_part() const { return reinterpret_cast<float *>(tc + T.part); }
+  int *ctr_p1() const { return reinterpret_cast<int *>(tc + T.ctr_p1); }
+  int *ctr_p2() const { return reinterpret_cast<int *>(tc + T.ctr_p2); }
+  int *ctr_up() const { return reinterpret_cast<int *>(tc + T.ctr_up); }
+  int *ctr_down() const { return reinterpret_cast<int *>(tc + T.ctr_down); }
 };
 
 pi_status get_ws(const pi_ffn *const *layers, int n, int B, void *ws, size_t ws_bytes, Ws *out) {
@@ -92,6 +140,16 @@ pi_status get_ws(const pi_ffn *const *layers, int n, int B, void *ws, size_t ws_
   if (G <= 0) return PI_ERR_CUDA;
   out->L = ws_layout(dmax, fmax, rmax, B, G);
   out->base = static_cast<char *>(ws);
+  out->tc = nullptr;
+  if (B >= kTcMinBatch) {
+    out->T = tc_layout(dmax, fmax, rmax, G);
+    if (out->T.total > ws_bytes) return PI_ERR_WORKSPACE;
+    const uintptr_t end = reinterpret_cast<uintptr_t>(ws) + ws_bytes;
+    const uintptr_t tc = (end - out->T.total) & ~(uintptr_t)255;
+    if (tc < reinterpret_cast<uintptr_t>(ws) + out->L.total) return PI_ERR_WORKSPACE;
+    out->tc = reinterpret_cast<char *>(tc);
+    return PI_OK;
+  }
   return out->L.total <= ws_bytes ? PI_OK : PI_ERR_WORKSPACE;
 }
 
@@ -294,6 +352,142 @@ pi_status run_ffn(const pi_ffn *h, const void *u, int B, float *out, int accumul
   return PI_OK;
 }
 
+// ---------------------------------------------------------------- tensor-core path (batch 16..32)
+namespace TC = pi::tc;
+
+// The tcgen05 kernels take fp16 predictors and fp16 or int4 weights (int4
+// rows in whole 256-element scale blocks) at 16 <= B <= 32.
+bool tc_ok(const pi_ffn *h, int B) {
+  const pi_ffn_desc &D = h->d;
+  if (B < kTcMinBatch || B > TC::kN || D.ptype != PI_W_F16) return false;
+  if (D.wtype == PI_W_F16) return true;
+  return D.wtype == PI_W_INT4G32 && D.d_model % 256 == 0;
+}
+
+template <typename KArg>
+cudaError_t launch_smem(void (*kern)(KArg), int G, int smem, bool *attr_done, cudaStream_t st, const KArg &arg) {
+  if (!*attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    *attr_done = true;
+  }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(G);
+  cfg.blockDim = dim3(TC::kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, arg);
+}
+
+template <int KIND, int WT, int ACT>
+cudaError_t ts_launch(const TC::TsArgs &a, int G, cudaStream_t st) {
+  static bool attr = false;
+  return launch_smem(TC::ts_gemm_kernel<KIND, WT, ACT>, G, TC::TsShape<KIND, WT, ACT>::SMEM, &attr, st, a);
+}
+
+template <int WT>
+cudaError_t down_launch(const TC::DownArgs &a, int G, cudaStream_t st) {
+  static bool attr = false;
+  return launch_smem(TC::ffn_down_kernel<WT>, G, TC::DownShape<WT>::SMEM, &attr, st, a);
+}
+
+cudaError_t tc_u_image(const pi_ffn *h, const void *u, int B, const Ws &w, cudaStream_t st) {
+  const int d = h->d.d_model;
+  const int total = TC::kN * ((d + 127) / 128) * 16;
+  return launch(TC::u_image_kernel, dim3(cdiv(total, 256)), dim3(256), st, (const __half *)u, B, d, w.uimg());
+}
+
+// steps 1-2 on tensor cores: u image, h = P1 u (hi/lo images), mask words, compaction
+pi_status run_predict_tc(const pi_ffn *h, const void *u, int B, int32_t *idx, int idx_stride, int32_t *count,
+                         const Ws &w, cudaStream_t st) {
+  const pi_ffn_desc &D = h->d;
+  const int G = w.L.G;
+  PI_CUDA(tc_u_image(h, u, B, w, st));
+  TC::TsArgs a{};
+  a.w0 = D.p1;
+  a.nrows = D.rank;
+  a.K = D.d_model;
+  a.img0 = w.uimg();
+  a.out0 = w.himg_hi();
+  a.out1 = w.himg_lo();
+  a.part = w.tc_part();
+  a.ctr = w.ctr_p1();
+  a.status = w.status();
+  a.B = B;
+  PI_CUDA((ts_launch<TC::K_P1, pi::W_F16, 0>(a, G, st)));
+  TC::TsArgs b{};
+  b.w0 = D.p2;
+  b.nrows = D.d_ffn;
+  b.K = D.rank;
+  b.img0 = w.himg_hi();
+  b.img1 = w.himg_lo();
+  b.bias = D.p_bias;
+  b.mask_out = w.mask();
+  b.nwords = h->nwords;
+  b.B = B;
+  b.part = w.tc_part();
+  b.ctr = w.ctr_p2();
+  b.status = w.status();
+  PI_CUDA((ts_launch<TC::K_P2, pi::W_F16, 0>(b, G, st)));
+  PI_CUDA(launch(pi::compact_kernel, dim3(B + 1), dim3(1024), st, (const uint32_t *)w.mask(), h->nwords, idx_stride, B,
+                 idx, count, w.uwords(), w.uprefix(), w.ulist(), w.ucount()));
+  return PI_OK;
+}
+
+// steps 3-4 on tensor cores over the union in the workspace; out (=, +=) y
+pi_status run_ffn_tc(const pi_ffn *h, const void *u, int B, float *out, int accumulate, bool u_ready, const Ws &w,
+                     cudaStream_t st) {
+  const pi_ffn_desc &D = h->d;
+  const int G = w.L.G;
+  if (!u_ready) PI_CUDA(tc_u_image(h, u, B, w, st));
+  TC::TsArgs a{};
+  a.w0 = D.w_up;
+  a.w1 = D.w_gate;
+  a.s0 = reinterpret_cast<const __half *>(D.s_up);
+  a.s1 = reinterpret_cast<const __half *>(D.s_gate);
+  a.rowlist = w.ulist();
+  a.rowcount = w.ucount();
+  a.K = D.d_model;
+  a.img0 = w.uimg();
+  a.bias = D.b_up;
+  a.mask = w.mask();
+  a.nwords = h->nwords;
+  a.B = B;
+  a.out0 = w.aimg();
+  a.part = w.tc_part();
+  a.ctr = w.ctr_up();
+  a.status = w.status();
+  const bool relu = D.act == PI_ACT_RELU;
+  cudaError_t e;
+  if (D.wtype == PI_W_F16)
+    e = relu ? ts_launch<TC::K_UP, pi::W_F16, pi::ACT_RELU>(a, G, st)
+             : ts_launch<TC::K_UP, pi::W_F16, pi::ACT_SWIGLU>(a, G, st);
+  else
+    e = relu ? ts_launch<TC::K_UP, pi::W_INT4, pi::ACT_RELU>(a, G, st)
+             : ts_launch<TC::K_UP, pi::W_INT4, pi::ACT_SWIGLU>(a, G, st);
+  PI_CUDA(e);
+  TC::DownArgs dn{};
+  dn.w = D.w_down_t;
+  dn.s = reinterpret_cast<const __half *>(D.s_down_t);
+  dn.rowlist = w.ulist();
+  dn.rowcount = w.ucount();
+  dn.d = D.d_model;
+  dn.B = B;
+  dn.aimg = w.aimg();
+  dn.y = out;
+  dn.accumulate = accumulate;
+  dn.part = w.tc_part();
+  dn.ctr = w.ctr_down();
+  dn.status = w.status();
+  PI_CUDA(D.wtype == PI_W_F16 ? down_launch<pi::W_F16>(dn, G, st) : down_launch<pi::W_INT4>(dn, G, st));
+  return PI_OK;
+}
+
 // ---------------------------------------------------------------- fused batch-1 path
 namespace F = pi::fused;
 
@@ -479,6 +673,7 @@ pi_status pi_workspace_size(const pi_ffn_t *layers, int n_layers, int max_batch,
   const int G = device_sm_count();
   if (G <= 0) return PI_ERR_CUDA;
   *bytes = ws_layout(dmax, fmax, rmax, max_batch, G).total;
+  if (max_batch >= kTcMinBatch) *bytes += tc_layout(dmax, fmax, rmax, G).total + 256;
   return PI_OK;
 }
 
@@ -498,6 +693,7 @@ pi_status pi_predict(pi_ffn_t h, const void *u, int B, int32_t *idx, int32_t *co
   Ws w;
   const pi_ffn *L[1] = {h};
   if ((s = get_ws(L, 1, B, ws, ws_bytes, &w)) != PI_OK) return s;
+  if (tc_ok(h, B)) return run_predict_tc(h, u, B, idx, h->d.d_ffn, count, w, (cudaStream_t)stream);
   return run_predict(h, u, B, idx, h->d.d_ffn, count, w, (cudaStream_t)stream);
 }
 
@@ -514,6 +710,7 @@ pi_status pi_sparse_ffn(pi_ffn_t h, const void *u, int B, const int32_t *idx, co
   if ((s = get_ws(L, 1, B, ws, ws_bytes, &w)) != PI_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
   if ((s = run_sets(h, idx, count, B, w, st)) != PI_OK) return s;
+  if (tc_ok(h, B)) return run_ffn_tc(h, u, B, y, (flags & PI_FFN_ACCUMULATE) ? 1 : 0, false, w, st);
   return run_ffn(h, u, B, y, (flags & PI_FFN_ACCUMULATE) ? 1 : 0, flags, w, st);
 }
 
@@ -532,6 +729,10 @@ pi_status pi_decode_ffn(pi_ffn_t h, const void *u, int B, float *y, int32_t *idx
   cudaStream_t st = (cudaStream_t)stream;
   const int acc = (flags & PI_FFN_ACCUMULATE) ? 1 : 0;
   if (fused_ok(h, B, w.L.G)) return run_fused(h, u, y, 0, acc, idx, count, flags, w, st);
+  if (tc_ok(h, B)) {
+    if ((s = run_predict_tc(h, u, B, idx, h->d.d_ffn, count, w, st)) != PI_OK) return s;
+    return run_ffn_tc(h, u, B, y, acc, true, w, st);
+  }
   if ((s = run_predict(h, u, B, idx, h->d.d_ffn, count, w, st)) != PI_OK) return s;
   return run_ffn(h, u, B, y, acc, flags, w, st);
 }
@@ -564,6 +765,11 @@ pi_status pi_decode_ffn_stack(const pi_ffn_t *layers, int L, float *x, int B, in
       continue;
     }
     PI_CUDA(launch(pi::rmsnorm_kernel, dim3(B), dim3(256), st, (const float *)x, d, w.u()));
+    if (tc_ok(layers[l], B)) {
+      if ((s = run_predict_tc(layers[l], w.u(), B, idx, fmax, cnt, w, st)) != PI_OK) return s;
+      if ((s = run_ffn_tc(layers[l], w.u(), B, x, 1, true, w, st)) != PI_OK) return s;
+      continue;
+    }
     if ((s = run_predict(layers[l], w.u(), B, idx, fmax, cnt, w, st)) != PI_OK) return s;
     if ((s = run_ffn(layers[l], w.u(), B, x, 1, flags, w, st)) != PI_OK) return s;
   }
