@@ -1,6 +1,7 @@
 // pi_ffn.cu -- C ABI of the predictor-gated sparse FFN decode library: host
 // validation, workspace layout and kernel dispatch.  The declarations and
 // argument contracts live in include/pi_ffn.h.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -18,6 +19,9 @@ struct pi_ffn {
   pi_ffn_desc d;
   int H;       // hot prefix rounded down to a multiple of 32
   int nwords;  // ceil(f / 32)
+  // TMA tensor maps of the tensor-core path (valid when tc_maps)
+  bool tc_maps;
+  CUtensorMap tm_p1, tm_p2, tm_up, tm_gate, tm_down, ts_up, ts_gate, ts_down;
 };
 
 namespace {
@@ -76,7 +80,7 @@ struct TcLayout {
 TcLayout tc_layout(int dmax, int fmax, int rmax, int G) {
   TcLayout L{};
   size_t o = 0;
-  const size_t step_img = (size_t)pi::tc::kStepImg;
+  const size_t step_img = (size_t)pi::tc::kImgStep / 16 * pi::tc::kBlk;
   L.uimg = o;
   o = align_up(o + (size_t)((dmax + 127) / 128) * step_img, 256);
   L.himg_hi = o;
@@ -97,6 +101,67 @@ TcLayout tc_layout(int dmax, int fmax, int rmax, int G) {
   o = align_up(o + (size_t)((dmax + pi::tc::kDownTileD - 1) / pi::tc::kDownTileD) * 4, 256);
   L.total = o;
   return L;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against the driver library); null when no driver is present.
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encoder() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !p) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// 2D map of a row-major matrix [rows x inner] of 1- or 2-byte elements, box
+// [box_rows x box_inner]; 128-byte swizzle when swz.  Outside reads are zero.
+bool map_2d(CUtensorMap *m, const void *base, bool fp16, uint64_t inner, uint64_t rows, uint32_t box_inner,
+            uint32_t box_rows, bool swz) {
+  EncodeTiledFn enc = encoder();
+  if (!enc) return false;
+  const uint64_t esz = fp16 ? 2 : 1;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {inner * esz};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t es[2] = {1, 1};
+  return enc(m, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base),
+             dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             swz ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Tensor maps of the tcgen05 kernels: fp16 predictor; fp16 weights, or int4
+// weights whose rows hold whole 256-element scale blocks.
+bool build_tc_maps(pi_ffn *h) {
+  const pi_ffn_desc &D = h->d;
+  if (D.ptype != PI_W_F16) return false;
+  const uint64_t d = D.d_model, f = D.d_ffn, r = D.rank;
+  bool ok = map_2d(&h->tm_p1, D.p1, true, d, r, 64, 128, true) && map_2d(&h->tm_p2, D.p2, true, r, f, 64, 128, true);
+  const bool swiglu = D.act == PI_ACT_SWIGLU;
+  if (D.wtype == PI_W_F16) {
+    ok = ok && map_2d(&h->tm_up, D.w_up, true, d, f, 64, 128, true) &&
+         (!swiglu || map_2d(&h->tm_gate, D.w_gate, true, d, f, 64, 128, true)) &&
+         map_2d(&h->tm_down, D.w_down_t, true, d, f, 64, 64, true);
+  } else if (D.wtype == PI_W_INT4G32 && d % 256 == 0) {
+    ok = ok && map_2d(&h->tm_up, D.w_up, false, d / 2, f, 128, 128, true) &&
+         map_2d(&h->ts_up, D.s_up, false, d / 16, f, 16, 128, false) &&
+         (!swiglu || (map_2d(&h->tm_gate, D.w_gate, false, d / 2, f, 128, 128, true) &&
+                      map_2d(&h->ts_gate, D.s_gate, false, d / 16, f, 16, 128, false))) &&
+         map_2d(&h->tm_down, D.w_down_t, false, d / 2, f, 128, 64, true) &&
+         map_2d(&h->ts_down, D.s_down_t, false, d / 16, f, 16, 64, false);
+  } else {
+    ok = false;
+  }
+  return ok;
 }
 
 constexpr int kTcMinBatch = 16;
@@ -356,12 +421,9 @@ pi_status run_ffn(const pi_ffn *h, const void *u, int B, float *out, int accumul
 namespace TC = pi::tc;
 
 // The tcgen05 kernels take fp16 predictors and fp16 or int4 weights (int4
-// rows in whole 256-element scale blocks) at 16 <= B <= 32.
+// rows in whole 256-element scale blocks; see build_tc_maps) at 16 <= B <= 32.
 bool tc_ok(const pi_ffn *h, int B) {
-  const pi_ffn_desc &D = h->d;
-  if (B < kTcMinBatch || B > TC::kN || D.ptype != PI_W_F16) return false;
-  if (D.wtype == PI_W_F16) return true;
-  return D.wtype == PI_W_INT4G32 && D.d_model % 256 == 0;
+  return B >= kTcMinBatch && B <= TC::kN && h->tc_maps && h->d.d_ffn <= TC::kMaxTiles * TC::kM;
 }
 
 template <typename KArg>
@@ -385,9 +447,9 @@ cudaError_t launch_smem(void (*kern)(KArg), int G, int smem, bool *attr_done, cu
 }
 
 template <int KIND, int WT, int ACT>
-cudaError_t ts_launch(const TC::TsArgs &a, int G, cudaStream_t st) {
+cudaError_t ts_launch(const TC::RowArgs &a, int G, cudaStream_t st) {
   static bool attr = false;
-  return launch_smem(TC::ts_gemm_kernel<KIND, WT, ACT>, G, TC::TsShape<KIND, WT, ACT>::SMEM, &attr, st, a);
+  return launch_smem(TC::row_gemm_kernel<KIND, WT, ACT>, G, TC::RowShape<KIND, WT, ACT>::SMEM, &attr, st, a);
 }
 
 template <int WT>
@@ -408,20 +470,20 @@ pi_status run_predict_tc(const pi_ffn *h, const void *u, int B, int32_t *idx, in
   const pi_ffn_desc &D = h->d;
   const int G = w.L.G;
   PI_CUDA(tc_u_image(h, u, B, w, st));
-  TC::TsArgs a{};
-  a.w0 = D.p1;
+  TC::RowArgs a{};
+  a.tm0 = h->tm_p1;
   a.nrows = D.rank;
   a.K = D.d_model;
   a.img0 = w.uimg();
   a.out0 = w.himg_hi();
   a.out1 = w.himg_lo();
+  a.B = B;
   a.part = w.tc_part();
   a.ctr = w.ctr_p1();
   a.status = w.status();
-  a.B = B;
   PI_CUDA((ts_launch<TC::K_P1, pi::W_F16, 0>(a, G, st)));
-  TC::TsArgs b{};
-  b.w0 = D.p2;
+  TC::RowArgs b{};
+  b.tm0 = h->tm_p2;
   b.nrows = D.d_ffn;
   b.K = D.rank;
   b.img0 = w.himg_hi();
@@ -445,13 +507,13 @@ pi_status run_ffn_tc(const pi_ffn *h, const void *u, int B, float *out, int accu
   const pi_ffn_desc &D = h->d;
   const int G = w.L.G;
   if (!u_ready) PI_CUDA(tc_u_image(h, u, B, w, st));
-  TC::TsArgs a{};
-  a.w0 = D.w_up;
-  a.w1 = D.w_gate;
-  a.s0 = reinterpret_cast<const __half *>(D.s_up);
-  a.s1 = reinterpret_cast<const __half *>(D.s_gate);
-  a.rowlist = w.ulist();
-  a.rowcount = w.ucount();
+  TC::RowArgs a{};
+  a.tm0 = h->tm_up;
+  a.tm1 = h->tm_gate;
+  a.ts0 = h->ts_up;
+  a.ts1 = h->ts_gate;
+  a.uwords = w.uwords();
+  a.nrows = D.d_ffn;
   a.K = D.d_model;
   a.img0 = w.uimg();
   a.bias = D.b_up;
@@ -472,10 +534,11 @@ pi_status run_ffn_tc(const pi_ffn *h, const void *u, int B, float *out, int accu
              : ts_launch<TC::K_UP, pi::W_INT4, pi::ACT_SWIGLU>(a, G, st);
   PI_CUDA(e);
   TC::DownArgs dn{};
-  dn.w = D.w_down_t;
-  dn.s = reinterpret_cast<const __half *>(D.s_down_t);
-  dn.rowlist = w.ulist();
-  dn.rowcount = w.ucount();
+  dn.tm = h->tm_down;
+  dn.ts = h->ts_down;
+  dn.uwords = w.uwords();
+  dn.nwords = h->nwords;
+  dn.f = D.d_ffn;
   dn.d = D.d_model;
   dn.B = B;
   dn.aimg = w.aimg();
@@ -653,6 +716,7 @@ pi_status pi_ffn_create(const pi_ffn_desc *desc, pi_ffn_t *out) {
   h->d = D;
   h->H = D.hot_prefix & ~31;
   h->nwords = (D.d_ffn + 31) / 32;
+  h->tc_maps = build_tc_maps(h);
   *out = h;
   return PI_OK;
 }

@@ -1,37 +1,41 @@
 // pi_tc.cuh -- tensor-core (tcgen05) path for token batches of 16..32.
 //
 // At batch >= 16 the union of the tokens' predicted sets covers nearly every
-// neuron, so each gathered block is a dense contraction (the 16..32 token
-// columns are the MMA's N).  Four persistent kernels run it, each on one CTA
-// per SM with a stream-K split of its (tile, K-step) work so that all SMs end
-// together:
+// neuron, so each 128-neuron block is a dense contraction with the 16..32
+// token columns as the MMA's N.  Four persistent kernels run the step, each
+// on one CTA per SM with a stream-K split of its (tile, K-step) units so that
+// all SMs end together:
 //
-//   pred_h  : h^T[r x N]  = P1 u^T              (A = P1 rows, K = d)
-//   pred_s  : s^T[f x N]  = P2 (h_hi + h_lo)^T  (A = P2 rows, K = r) + bias,
-//             thresholded to the per-token mask words
-//   ffn_up  : a^T[U x N]  = act(W_up/gate[union] u^T), zero where the token
-//             did not predict the neuron        (A = gathered rows, K = d)
-//   ffn_down: y^T[d x N]  = W2T[union]^T a^T    (A = gathered W2T rows, MN-major)
+//   pred_h  : h^T[r x N]  = P1 u^T               (A = P1, K = d)
+//   pred_s  : s^T[f x N]  = P2 (h_hi + h_lo)^T   (A = P2, K = r) + bias,
+//             thresholded into the per-token mask words
+//   ffn_up  : a^T         = act(W_up/gate u^T) on every 128-neuron tile that
+//             holds a predicted neuron of some token; zero where the token
+//             did not predict the neuron        (A = weight rows, K = d)
+//   ffn_down: y^T[d x N]  = W2T^T a^T over those tiles (A = W2T, MN-major)
 //
-// The three "row" kernels use one template (ts_gemm_kernel): a producer warp
-// copies 128 rows x 128 K of row data into a shared-memory ring with
-// cp.async; eight worker warps move it (dequantising int4) into tensor memory
-// as the MMA's A operand; one thread issues tcgen05.mma with the token image
-// (B operand) in shared memory; the worker warps also run the epilogue.  The
-// down kernel keeps A in shared memory (the d positions are the MMA's M, so a
-// neuron row lands as 16-byte MN-major pieces).
+// Row data moves by TMA (2D tensor maps, one 16 KB box of 128 rows per
+// copy).  fp16 boxes land 128B-swizzled, which is the canonical UMMA layout,
+// so the MMA reads them in place.  int4 boxes (packed nibbles + the group
+// scales) are dequantised by eight worker warps into tensor memory (A operand
+// of the MMA) for the up/gate GEMM, or into a canonical shared-memory tile
+// for the down GEMM.  One thread issues the MMAs; the worker warps also run
+// the epilogues.
 //
-// Token operands are stored as "images": per 16-deep K block, 1 KB holding
-// the 32 token rows in the canonical no-swizzle K-major UMMA layout (core
-// matrices of 8 tokens x 8 K, 16-byte rows).  Padding tokens and K beyond the
-// row length are zero, so padded MMA work adds exact zeros.
+// Token operands are "images": per 16-deep K block, 1 KB holding the 32 token
+// rows in the canonical no-swizzle K-major layout (core matrices of 8 tokens
+// x 8 K, 16-byte rows).  Padding tokens and K beyond the row are zero, and
+// TMA fills rows or columns outside a matrix with zeros, so padded MMA work
+// adds exact zeros.
 //
-// Stream-K: a kernel's W = tiles x steps units are split into G contiguous
-// spans.  A tile whose steps span several CTAs is finished by the last CTA to
-// arrive (per-tile counter): it adds the pieces' fp32 partials in K order, so
-// the result does not depend on timing.  Counters reset themselves.
+// Stream-K: a kernel's W = tiles x steps units are split into contiguous
+// spans over min(G, W) CTAs.  A tile whose steps span several CTAs is
+// finished by the last CTA to arrive (per-tile counter): it adds the pieces'
+// fp32 partials in K order, so the result does not depend on timing.
+// Counters reset themselves.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_fp16.h>
 #include <stdint.h>
 
@@ -42,15 +46,16 @@ namespace tc {
 
 constexpr int kN = 32;        // MMA N: token columns (batches of 16..32 are zero-padded)
 constexpr int kM = 128;       // MMA M: rows of a tile
-constexpr int kStepK = 128;   // K per pipeline step of the row kernels
 constexpr int kBlk = 1024;    // bytes of one 16-deep K block of a token image
-constexpr int kStepImg = 8 * kBlk;
 constexpr int kThreads = 320; // warp 0 producer, warp 1 MMA issuer, warps 2..9 workers
 constexpr int kWorkerThreads = 256;
-constexpr int kSmemBudget = 212 * 1024;
+constexpr int kSmemBudget = 216 * 1024;
 constexpr int kPartFloats = 128 * 64;  // largest per-piece partial (floats)
 constexpr int kDownTileD = 256;        // d positions per down-projection tile (two M=128 MMAs)
-constexpr int kDownStepK = 64;         // union positions per down-projection step
+constexpr int kDownStepK = 64;         // neurons per down-projection step
+constexpr int kMaxTiles = 1024;        // 128-neuron tiles the ffn kernels can list (d_ffn <= 131072)
+constexpr int kImgStep = 128;          // token images are padded to a multiple of 128 in K
+constexpr uint32_t kSw128 = 2;         // UMMA descriptor layout code of the 128-byte swizzle
 constexpr unsigned long long kWaitNs = 2000000000ull;
 
 enum Kind { K_P1 = 0, K_P2 = 1, K_UP = 2 };
@@ -112,15 +117,15 @@ PI_DEV bool workers_bar(uint64_t *b, unsigned &phase, volatile int *abort_flag, 
   return ok;
 }
 
-// 16-byte cp.async; src_bytes 0 fills the destination with zeros
-PI_DEV void cp16(uint32_t dst, const void *src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+// 2D TMA tile load of the box at element coordinates (x, y) of a tensor map
+// (a kernel parameter); rows or columns outside the tensor read as zero
+PI_DEV void tma_load_2d(uint32_t dst, const CUtensorMap *tm, int x, int y, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(su32(bar))
+      : "memory");
 }
-// arrive on b once all earlier cp.async of this thread have landed
-PI_DEV void cp_arrive(uint64_t *b) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(su32(b)) : "memory");
-}
-PI_DEV void cp_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 PI_DEV void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint64_t *bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
@@ -142,10 +147,11 @@ PI_DEV void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
 
-// UMMA shared-memory descriptor, no swizzle: start, leading and stride byte offsets
-PI_DEV uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+// UMMA shared-memory descriptor: start, leading and stride byte offsets,
+// layout (0: no swizzle, kSw128: 128-byte swizzle with 1024-byte aligned atoms)
+PI_DEV uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout = 0) {
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46);
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46) | ((uint64_t)layout << 61);
 }
 // instruction descriptor of kind::f16: fp16 A and B, fp32 accumulator, M x N
 __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int a_mn, int b_mn) {
@@ -237,7 +243,7 @@ __global__ void __launch_bounds__(256) u_image_kernel(const __half *__restrict__
                                                       unsigned char *__restrict__ img) {
   pdl_wait();
   pdl_launch_dependents();
-  const int nblk = (d + kStepK - 1) / kStepK * 8;
+  const int nblk = (d + kImgStep - 1) / kImgStep * 8;
   const int per_tok = nblk * 2;  // 16-byte pieces per token row of the image
   const int total = kN * per_tok;
   for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < total; c += gridDim.x * blockDim.x) {
@@ -250,70 +256,28 @@ __global__ void __launch_bounds__(256) u_image_kernel(const __half *__restrict__
   }
 }
 
-// ---------------------------------------------------------------- row GEMM (A in tensor memory)
-struct TsArgs {
-  const void *w0, *w1;           // row data of matrix 0 / 1 ([rows x K] fp16, or packed int4)
-  const __half *s0, *s1;         // int4 group scales [rows x K/32]
-  const int32_t *rowlist;        // ffn_up: union position -> neuron id
-  const int32_t *rowcount;       // ffn_up: device union size U
-  int nrows;                     // number of rows when rowcount is null
-  int K;                         // row length (elements)
-  const unsigned char *img0;     // B operand image (u, or h_hi)
-  const unsigned char *img1;     // pred_s: h_lo image
-  const float *bias;             // pred_s: predictor bias; ffn_up ReLU: b_up
-  const uint32_t *mask;          // ffn_up: per-token mask words [B x nwords]
-  uint32_t *mask_out;            // pred_s: per-token mask words [B x nwords]
-  int nwords, B;
-  unsigned char *out0, *out1;    // pred_h: h_hi / h_lo images; ffn_up: a image
-  float *part;                   // stream-K partials [G x 2 x kPartFloats]
-  int *ctr;                      // per-tile arrival counters (zero between launches)
-  int *status;
-};
-
-struct TsCtrl {
-  uint64_t full[6], img_full[6], empty[6], img_empty[6];
+// ---------------------------------------------------------------- shared pieces
+struct TcCtrl {
+  uint64_t full[6], empty[6];
   uint64_t afull[2], afree[2], accfull[2], accfree[2];
   uint64_t wbar;  // the 256 worker threads' barrier (stream-K fix-up)
   uint32_t tmem;
   int abort_flag;
   int is_last;
-  int rows[kM];   // producer: row ids of the current tile / step (-1: padding)
+  int n_tiles;    // tiles listed in tlist
+  int wcnt[kThreads / 32];
+  int tlist[kMaxTiles];  // ffn kernels: 128-neuron tiles holding a predicted neuron
 };
-constexpr int kCtrlBytes = 1024;
-static_assert(sizeof(TsCtrl) <= kCtrlBytes, "control block");
+constexpr int kCtrlBytes = 5120;
+static_assert(sizeof(TcCtrl) <= kCtrlBytes, "control block");
 
-template <int KIND, int WT, int ACT>
-struct TsShape {
-  static constexpr int NMAT = (KIND == K_UP && ACT == ACT_SWIGLU) ? 2 : 1;
-  static constexpr int NIMG = KIND == K_P2 ? 2 : 1;
-  static constexpr bool Q4 = WT == W_INT4;
-  // staging row pitch per matrix for one step: int4 64 B packed + 16 B scales,
-  // fp16 256 B + 16 B pad (the pad spreads rows over the banks)
-  static constexpr int ROWB = Q4 ? 80 : 272;
-  static constexpr int SLOTB = NMAT * kM * ROWB;
-  static constexpr int IMGB = NIMG * kStepImg;
-  static constexpr int NSLOT_FIT = kSmemBudget / (SLOTB + IMGB);
-  static constexpr int NSLOT = NSLOT_FIT > 6 ? 6 : NSLOT_FIT;
-  static constexpr int IMG_OFF = 0;
-  static constexpr int STAGE_OFF = NSLOT * IMGB;
-  static constexpr int CTRL_OFF = STAGE_OFF + NSLOT * SLOTB;
-  static constexpr int SMEM = CTRL_OFF + kCtrlBytes;
-  static constexpr int ACC_COLS = NMAT * kN;  // per accumulator buffer
-  static constexpr int A_COLS = NMAT * 64;    // per A buffer (128 K of fp16 pairs)
-  static constexpr uint32_t TMEM_COLS = 512;
-  static_assert(NSLOT >= 2, "ring too shallow");
-  static_assert(SMEM <= 227 * 1024, "shared memory");
-  static_assert(2 * ACC_COLS + 2 * A_COLS <= (int)TMEM_COLS, "tensor memory");
-};
-
-
+// empty_count: arrivals that free a ring slot (1: the MMA's commit; 9: the
+// 8 worker warps that read the slot and the MMA's commit)
 template <int NSLOT>
-PI_DEV void ctrl_init(TsCtrl &C) {
+PI_DEV void ctrl_init(TcCtrl &C, unsigned empty_count) {
   for (int s = 0; s < NSLOT; ++s) {
-    mbar_init(&C.full[s], 32);      // the producer warp's cp.async arrivals
-    mbar_init(&C.img_full[s], 1);   // expect_tx of the image bulk copy
-    mbar_init(&C.empty[s], 8);      // the 8 worker warps
-    mbar_init(&C.img_empty[s], 1);  // MMA commit
+    mbar_init(&C.full[s], 1);  // the producer's expect_tx; TMA completes the bytes
+    mbar_init(&C.empty[s], empty_count);
   }
   for (int b = 0; b < 2; ++b) {
     mbar_init(&C.afull[b], 8);
@@ -327,14 +291,42 @@ PI_DEV void ctrl_init(TsCtrl &C) {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
+// All threads: list the 128-neuron tiles that hold a set bit of the union
+// words (4 words per tile), in ascending order, into C.tlist / C.n_tiles.
+PI_DEV void list_tiles(TcCtrl &C, const uint32_t *uwords, int nwords, int n_all) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  int base = 0;
+  for (int t0 = 0; t0 < n_all; t0 += kThreads) {
+    const int t = t0 + tid;
+    bool act = false;
+    if (t < n_all) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (4 * t + k < nwords) act |= __ldg(uwords + 4 * t + k) != 0u;
+    }
+    const unsigned bal = __ballot_sync(0xffffffffu, act);
+    if (lane == 0) C.wcnt[warp] = __popc(bal);
+    __syncthreads();
+    int off = base;
+    for (int w = 0; w < warp; ++w) off += C.wcnt[w];
+    if (act) C.tlist[off + __popc(bal & ((1u << lane) - 1u))] = t;
+    int tot = 0;
+    for (int w = 0; w < kThreads / 32; ++w) tot += C.wcnt[w];
+    base += tot;
+    __syncthreads();
+  }
+  if (tid == 0) C.n_tiles = base;
+  __syncthreads();
+}
+
 // Stream-K fix-up for one worker thread's NV accumulator values of a piece
 // that does not cover its whole tile (G: the CTAs the units were split
-// over).  Publishes the piece; the CTA whose
-// piece arrives last sums all pieces in K order into v and returns true.
-// *ok turns false when a bounded wait gave up.
+// over).  Publishes the piece; the CTA whose piece arrives last sums all
+// pieces in K order into v and returns true.  *ok turns false when a bounded
+// wait gave up.
 template <int NV>
 PI_DEV bool stream_k_finish(float (&v)[NV], float *part, int *ctr, int tile, long long SK, long long W, int G,
-                            int cta, long long u0, int w, int lane, TsCtrl &C, unsigned &wphase,
+                            int cta, long long u0, int w, int lane, TcCtrl &C, unsigned &wphase,
                             volatile int *abort_flag, int *status, bool *ok) {
   const int slot = (int)(u0 / SK) == tile ? 0 : 1;
   float *mine = part + ((size_t)cta * 2 + slot) * kPartFloats;
@@ -379,31 +371,71 @@ PI_DEV bool stream_k_finish(float (&v)[NV], float *part, int *ctr, int tile, lon
   return true;
 }
 
-// Waits for the issuer's last commit (all MMAs done), then releases tensor memory.
-PI_DEV void teardown(TsCtrl &C, const Span &sp, int warp, int lane, uint32_t tmem, uint32_t ncols,
-                     volatile int *abort_flag, int *status) {
-  if (warp == 1 && lane == 0) {
-    const long long n_steps = sp.u1 - sp.u0;
-    if (n_steps > 0 && !*abort_flag) {
-      const long long il = n_steps - 1;
-      mbar_wait(&C.afree[il & 1], (unsigned)((il >> 1) & 1), abort_flag, status);
-    }
-  }
+// Releases tensor memory.  Every MMA has finished by then: the workers wait
+// for the commit that follows the last MMA of each piece, the last piece
+// included (a CTA that gave up on a bounded wait skips that guarantee).
+PI_DEV void teardown(int warp, uint32_t tmem, uint32_t ncols) {
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, ncols);
 }
 
+// ---------------------------------------------------------------- row GEMMs: pred_h, pred_s, ffn_up
+struct RowArgs {
+  CUtensorMap tm0, tm1;         // row data of matrix 0 / 1: fp16 [rows x K] (box 64 x 128) or
+                                // packed int4 bytes [rows x K/2] (box 128 x 128)
+  CUtensorMap ts0, ts1;         // int4 scale bytes [rows x K/16] (box 16 x 128)
+  const uint32_t *uwords;       // ffn_up: union mask words (a tile runs when one of its 4 words is set)
+  int nrows;                    // rows of the matrices
+  int K;                        // row length (elements)
+  const unsigned char *img0;    // B operand image (u, or h_hi)
+  const unsigned char *img1;    // pred_s: h_lo image
+  const float *bias;            // pred_s: predictor bias; ffn_up ReLU: b_up
+  const uint32_t *mask;         // ffn_up: per-token mask words [B x nwords]
+  uint32_t *mask_out;           // pred_s: per-token mask words [B x nwords]
+  int nwords, B;
+  unsigned char *out0, *out1;   // pred_h: h_hi / h_lo images; ffn_up: a image
+  float *part;                  // stream-K partials [G x 2 x kPartFloats]
+  int *ctr;                     // per-tile arrival counters (zero between launches)
+  int *status;
+};
+
 template <int KIND, int WT, int ACT>
-__global__ void __launch_bounds__(kThreads, 1) ts_gemm_kernel(const TsArgs a) {
-  using S = TsShape<KIND, WT, ACT>;
-  extern __shared__ __align__(1024) unsigned char smem[];
-  TsCtrl &C = *reinterpret_cast<TsCtrl *>(smem + S::CTRL_OFF);
+struct RowShape {
+  static constexpr int NMAT = (KIND == K_UP && ACT == ACT_SWIGLU) ? 2 : 1;
+  static constexpr int NIMG = KIND == K_P2 ? 2 : 1;
+  static constexpr bool Q4 = WT == W_INT4;
+  static constexpr int STEPK = Q4 ? 256 : 64;       // K per unit
+  static constexpr int ABOX = 16384;                // one box: 128 rows x 128 bytes
+  static constexpr int SBOX = Q4 ? 2048 : 0;        // int4 scales: 128 rows x 16 bytes
+  static constexpr int IMGB = NIMG * (STEPK / 16) * kBlk;
+  static constexpr int SC_OFF = NMAT * ABOX;
+  static constexpr int IMG_OFF = NMAT * (ABOX + SBOX);
+  static constexpr int SLOTB = (IMG_OFF + IMGB + 1023) / 1024 * 1024;
+  static constexpr int NSLOT_FIT = kSmemBudget / SLOTB;
+  static constexpr int NSLOT = NSLOT_FIT > 6 ? 6 : NSLOT_FIT;
+  static constexpr int TX = IMG_OFF + IMGB;         // bytes landing per unit
+  static constexpr int CTRL_OFF = NSLOT * SLOTB;
+  static constexpr int SMEM = CTRL_OFF + kCtrlBytes + 1024;  // + alignment slack
+  static constexpr int ACC_COLS = NMAT * kN;        // per accumulator buffer
+  static constexpr int A_COLS = NMAT * 64;          // int4: per tensor-memory A buffer (128 K)
+  static constexpr uint32_t TMEM_COLS = Q4 ? 512 : 128;
+  static_assert(NSLOT >= 2, "ring too shallow");
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+  static_assert(2 * ACC_COLS + (Q4 ? 2 * A_COLS : 0) <= (int)TMEM_COLS, "tensor memory");
+};
+
+template <int KIND, int WT, int ACT>
+__global__ void __launch_bounds__(kThreads, 1) row_gemm_kernel(const __grid_constant__ RowArgs a) {
+  using S = RowShape<KIND, WT, ACT>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  TcCtrl &C = *reinterpret_cast<TcCtrl *>(smem + S::CTRL_OFF);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, cta = blockIdx.x;
 
-  if (tid == 0) ctrl_init<S::NSLOT>(C);
+  if (tid == 0) ctrl_init<S::NSLOT>(C, S::Q4 ? 9u : 1u);
   if (warp == 1) tmem_alloc(&C.tmem, S::TMEM_COLS);
   tc_fence_before();
   __syncthreads();
@@ -414,94 +446,54 @@ __global__ void __launch_bounds__(kThreads, 1) ts_gemm_kernel(const TsArgs a) {
   pdl_wait();
   pdl_launch_dependents();
 
-  const int nrows = a.rowcount ? *a.rowcount : a.nrows;
-  const long long T = (nrows + kM - 1) / kM;
-  const long long SK = (a.K + kStepK - 1) / kStepK;
+  const int T_all = (a.nrows + kM - 1) / kM;
+  if (KIND == K_UP) {
+    list_tiles(C, a.uwords, a.nwords, T_all);
+  } else if (tid == 0) {
+    C.n_tiles = T_all;
+  }
+  __syncthreads();
+  const long long T = C.n_tiles;
+  const long long SK = (a.K + S::STEPK - 1) / S::STEPK;
   const long long W = T * SK;
   // stream-K over min(G, W) CTAs so that every CTA taking part owns a unit
   const int Gs = (int)(W < G ? W : G);
   const Span sp = cta < Gs ? span_of(W, Gs, cta) : Span{0, 0};
+  auto tile_of = [&](long long j) -> int { return KIND == K_UP ? C.tlist[j] : (int)j; };
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    const size_t rowB = S::Q4 ? (size_t)a.K / 2 : (size_t)a.K * 2;
-    const size_t srowB = (size_t)a.K / 16;  // int4 scale bytes per row
-    long long cur_tile = -1;
-    long long i = 0;
-    for (long long u = sp.u0; u < sp.u1; ++u, ++i) {
-      const int s = (int)(i % S::NSLOT);
-      const unsigned ph = (unsigned)((i / S::NSLOT) & 1);
-      if (i >= S::NSLOT) {
-        if (!mbar_wait_warp(&C.empty[s], ph ^ 1u, abort_flag, a.status)) break;
-        if (!mbar_wait_warp(&C.img_empty[s], ph ^ 1u, abort_flag, a.status)) break;
-      }
-      const long long tile = u / SK;
-      const int step = (int)(u % SK);
-      if (tile != cur_tile) {
-        cur_tile = tile;
-        __syncwarp();
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const long long p = tile * kM + lane + 32 * j;
-          C.rows[lane + 32 * j] = p < nrows ? (a.rowlist ? __ldg(a.rowlist + p) : (int)p) : -1;
-        }
-        __syncwarp();
-      }
-      if (lane == 0) {
-        mbar_expect_tx(&C.img_full[s], S::IMGB);
-        const uint32_t d0 = su32(smem + S::IMG_OFF + s * S::IMGB);
-        bulk_g2s(d0, a.img0 + (size_t)step * kStepImg, kStepImg, &C.img_full[s]);
-        if (S::NIMG == 2) bulk_g2s(d0 + kStepImg, a.img1 + (size_t)step * kStepImg, kStepImg, &C.img_full[s]);
-      }
-      // rows as 16-byte pieces, zero-filled beyond the row and for padding rows
-      const uint32_t st0 = su32(smem + S::STAGE_OFF + s * S::SLOTB);
-      const int k0 = step * kStepK;
-#pragma unroll
-      for (int mat = 0; mat < S::NMAT; ++mat) {
-        const unsigned char *wb = reinterpret_cast<const unsigned char *>(mat == 0 ? a.w0 : a.w1);
-        const uint32_t sm0 = st0 + mat * kM * S::ROWB;
-        if constexpr (S::Q4) {
-          // 5 pieces per row: 4 x 16 B of packed nibbles (128 elements) and
-          // the 16-byte block of the 8 group scales of the enclosing 256 elements
-          const unsigned char *sb = reinterpret_cast<const unsigned char *>(mat == 0 ? a.s0 : a.s1);
-#pragma unroll 4
-          for (int qq = lane; qq < kM * 5; qq += 32) {
-            const int m = qq / 5, c = qq - m * 5;
-            const int rid = C.rows[m];
-            const uint32_t dst = sm0 + m * S::ROWB + c * 16;
-            if (c < 4) {
-              const bool ok = rid >= 0 && k0 + c * 32 < a.K;
-              cp16(dst, wb + (ok ? (size_t)rid * rowB + (size_t)k0 / 2 + c * 16 : 0), ok ? 16u : 0u);
-            } else {
-              const bool ok = rid >= 0;
-              cp16(dst, sb + (ok ? (size_t)rid * srowB + (size_t)(k0 / 256) * 16 : 0), ok ? 16u : 0u);
-            }
-          }
-        } else {
-#pragma unroll 4
-          for (int qq = lane; qq < kM * 16; qq += 32) {
-            const int m = qq >> 4, c = qq & 15;
-            const int rid = C.rows[m];
-            const bool ok = rid >= 0 && k0 + c * 8 < a.K;
-            cp16(sm0 + m * S::ROWB + c * 16, wb + (ok ? (size_t)rid * rowB + (size_t)(k0 + c * 8) * 2 : 0),
-                 ok ? 16u : 0u);
-          }
-        }
-      }
-      cp_arrive(&C.full[s]);
-    }
-    cp_wait_all();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ producer (one lane)
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_f16(kM, kN, 0, 0);
+      long long i = 0;
+      for (long long u = sp.u0; u < sp.u1; ++u, ++i) {
+        const int s = (int)(i % S::NSLOT);
+        const unsigned ph = (unsigned)((i / S::NSLOT) & 1);
+        if (i >= S::NSLOT && !mbar_wait(&C.empty[s], ph ^ 1u, abort_flag, a.status)) break;
+        const int row0 = tile_of(u / SK) * kM;
+        const int k0 = (int)(u % SK) * S::STEPK;
+        unsigned char *slot = smem + s * S::SLOTB;
+        mbar_expect_tx(&C.full[s], S::TX);
+#pragma unroll
+        for (int mat = 0; mat < S::NMAT; ++mat) {
+          tma_load_2d(su32(slot + mat * S::ABOX), mat == 0 ? &a.tm0 : &a.tm1, S::Q4 ? k0 / 2 : k0, row0, &C.full[s]);
+          if constexpr (S::Q4)
+            tma_load_2d(su32(slot + S::SC_OFF + mat * S::SBOX), mat == 0 ? &a.ts0 : &a.ts1, k0 / 16, row0, &C.full[s]);
+        }
+        const size_t ib = (size_t)(k0 / 16) * kBlk;
+        bulk_g2s(su32(slot + S::IMG_OFF), a.img0 + ib, (S::STEPK / 16) * kBlk, &C.full[s]);
+        if (S::NIMG == 2)
+          bulk_g2s(su32(slot + S::IMG_OFF + (S::STEPK / 16) * kBlk), a.img1 + ib, (S::STEPK / 16) * kBlk, &C.full[s]);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (one lane)
+    if (lane == 0) {
       long long i = 0;
       int piece = -1;
       for (long long u = sp.u0; u < sp.u1; ++u, ++i) {
         const int s = (int)(i % S::NSLOT);
         const unsigned ph = (unsigned)((i / S::NSLOT) & 1);
-        const int b = (int)(i & 1);
-        const unsigned bph = (unsigned)((i >> 1) & 1);
         const bool first = (u == sp.u0) || (u % SK == 0);
         if (first) {
           ++piece;
@@ -509,36 +501,55 @@ __global__ void __launch_bounds__(kThreads, 1) ts_gemm_kernel(const TsArgs a) {
               !mbar_wait(&C.accfree[piece & 1], (unsigned)(((piece >> 1) & 1) ^ 1), abort_flag, a.status))
             break;
         }
-        if (!mbar_wait(&C.afull[b], bph, abort_flag, a.status)) break;
-        if (!mbar_wait(&C.img_full[s], ph, abort_flag, a.status)) break;
+        if (!mbar_wait(&C.full[s], ph, abort_flag, a.status)) break;
         tc_fence_after();
         const uint32_t acc = tmem + (uint32_t)((piece & 1) * S::ACC_COLS);
-        const uint32_t abuf = tmem + (uint32_t)(2 * S::ACC_COLS + b * S::A_COLS);
-        const uint32_t img = su32(smem + S::IMG_OFF + s * S::IMGB);
+        const uint32_t slot = su32(smem + s * S::SLOTB);
+        constexpr uint32_t idesc = idesc_f16(kM, kN, 0, 0);
+        if constexpr (!S::Q4) {
+          // A straight from the swizzled TMA box: 16 K = 32 bytes along the 128-byte rows
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+          for (int j = 0; j < 4; ++j)
 #pragma unroll
-          for (int mat = 0; mat < S::NMAT; ++mat) {
+            for (int mat = 0; mat < S::NMAT; ++mat)
 #pragma unroll
-            for (int nb = 0; nb < S::NIMG; ++nb) {
-              const uint64_t bd = sdesc(img + nb * kStepImg + j * kBlk, 128, 256);
-              const uint32_t accum = (first && j == 0 && nb == 0) ? 0u : 1u;
-              mma_ts(acc + mat * kN, abuf + mat * 64 + j * 8, bd, idesc, accum);
-            }
+              for (int nb = 0; nb < S::NIMG; ++nb) {
+                const uint64_t ad = sdesc(slot + mat * S::ABOX + j * 32, 16, 1024, kSw128);
+                const uint64_t bd = sdesc(slot + S::IMG_OFF + nb * 4 * kBlk + j * kBlk, 128, 256);
+                mma_ss(acc + mat * kN, ad, bd, idesc, (first && j == 0 && nb == 0) ? 0u : 1u);
+              }
+          mma_commit(&C.empty[s]);
+        } else {
+          // two 128-K halves, each dequantised by the workers into a tensor-memory A buffer
+#pragma unroll 1
+          for (int sub = 0; sub < 2; ++sub) {
+            const long long ia = 2 * i + sub;
+            const int b = (int)(ia & 1);
+            if (!mbar_wait(&C.afull[b], (unsigned)((ia >> 1) & 1), abort_flag, a.status)) break;
+            tc_fence_after();
+            const uint32_t abuf = tmem + (uint32_t)(2 * S::ACC_COLS + b * S::A_COLS);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+#pragma unroll
+              for (int mat = 0; mat < S::NMAT; ++mat) {
+                const uint64_t bd = sdesc(slot + S::IMG_OFF + (sub * 8 + j) * kBlk, 128, 256);
+                mma_ts(acc + mat * kN, abuf + mat * 64 + j * 8, bd, idesc, (first && sub == 0 && j == 0) ? 0u : 1u);
+              }
+            mma_commit(&C.afree[b]);
           }
+          if (*abort_flag) break;
+          mma_commit(&C.empty[s]);
         }
-        mma_commit(&C.afree[b]);
-        mma_commit(&C.img_empty[s]);
         const bool last = (u + 1 == sp.u1) || ((u + 1) % SK == 0);
         if (last) mma_commit(&C.accfull[piece & 1]);
       }
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ workers: A operand + epilogue
+    // ------------------------------------------------------------ workers: int4 A operand + epilogues
     const int w = warp - 2;       // 0..7
     const int q = warp & 3;       // tensor-memory lane quarter of this warp
-    const int h = w >> 2;         // K half of a step; token half of the epilogue
+    const int h = w >> 2;         // K half of a dequant step; token half of the epilogue
     const int m = q * 32 + lane;  // row within the tile
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
     unsigned wphase = 0;
@@ -547,57 +558,56 @@ __global__ void __launch_bounds__(kThreads, 1) ts_gemm_kernel(const TsArgs a) {
     int piece = -1;
     long long piece_u0 = sp.u0;
     for (long long u = sp.u0; u < sp.u1 && ok; ++u, ++i) {
-      const int s = (int)(i % S::NSLOT);
-      const unsigned ph = (unsigned)((i / S::NSLOT) & 1);
-      const int b = (int)(i & 1);
-      const unsigned bph = (unsigned)((i >> 1) & 1);
-      const long long tile = u / SK;
-      const int step = (int)(u % SK);
-      if ((u == sp.u0) || (step == 0)) {
+      const long long j_tile = u / SK;
+      if ((u == sp.u0) || (u % SK == 0)) {
         ++piece;
         piece_u0 = u;
       }
-      if (!mbar_wait_warp(&C.full[s], ph, abort_flag, a.status)) break;
-      if (i >= 2 && !mbar_wait_warp(&C.afree[b], bph ^ 1u, abort_flag, a.status)) break;
-      const unsigned char *st = smem + S::STAGE_OFF + s * S::SLOTB;
-      const uint32_t acol = lane_base + (uint32_t)(2 * S::ACC_COLS + b * S::A_COLS + h * 32);
-#pragma unroll
-      for (int mat = 0; mat < S::NMAT; ++mat) {
-        const unsigned char *row = st + mat * kM * S::ROWB + m * S::ROWB;
-        uint32_t v[32];
-        if constexpr (S::Q4) {
-          const uint4 p0 = *reinterpret_cast<const uint4 *>(row + h * 32);
-          const uint4 p1 = *reinterpret_cast<const uint4 *>(row + h * 32 + 16);
-          const uint32_t sc = *reinterpret_cast<const uint32_t *>(row + 64 + ((step & 1) * 4 + h * 2) * 2);
-          const __half s_lo = __ushort_as_half((unsigned short)(sc & 0xFFFFu));
-          const __half s_hi = __ushort_as_half((unsigned short)(sc >> 16));
-          const __half2 sA = __halves2half2(s_lo, s_lo), sB = __halves2half2(s_hi, s_hi);
-          const uint32_t wds[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-#pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            uint32_t o[4];
-            q8_to_h4(wds[t], t < 4 ? sA : sB, o);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) v[t * 4 + c] = o[c];
+      if constexpr (S::Q4) {
+        const int s = (int)(i % S::NSLOT);
+        const unsigned ph = (unsigned)((i / S::NSLOT) & 1);
+        if (!mbar_wait_warp(&C.full[s], ph, abort_flag, a.status)) break;
+        const unsigned char *slot = smem + s * S::SLOTB;
+        bool fine = true;
+#pragma unroll 1
+        for (int sub = 0; sub < 2 && fine; ++sub) {
+          const long long ia = 2 * i + sub;
+          const int b = (int)(ia & 1);
+          if (ia >= 2 && !mbar_wait_warp(&C.afree[b], (unsigned)(((ia >> 1) & 1) ^ 1), abort_flag, a.status)) {
+            fine = false;
+            break;
           }
-        } else {
+          const uint32_t acol = lane_base + (uint32_t)(2 * S::ACC_COLS + b * S::A_COLS + h * 32);
 #pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            const uint4 p = *reinterpret_cast<const uint4 *>(row + h * 128 + t * 16);
-            v[t * 4 + 0] = p.x;
-            v[t * 4 + 1] = p.y;
-            v[t * 4 + 2] = p.z;
-            v[t * 4 + 3] = p.w;
+          for (int mat = 0; mat < S::NMAT; ++mat) {
+            // packed row m of the swizzled box: 16-byte chunk c sits at (c ^ (m % 8)) * 16
+            const unsigned char *row = slot + mat * S::ABOX + m * 128;
+            const int c0 = sub * 4 + h * 2;
+            const uint4 p0 = *reinterpret_cast<const uint4 *>(row + ((c0 ^ (m & 7)) << 4));
+            const uint4 p1 = *reinterpret_cast<const uint4 *>(row + (((c0 + 1) ^ (m & 7)) << 4));
+            const uint32_t sc = *reinterpret_cast<const uint32_t *>(slot + S::SC_OFF + mat * S::SBOX + m * 16 + c0 * 2);
+            const __half s_lo = __ushort_as_half((unsigned short)(sc & 0xFFFFu));
+            const __half s_hi = __ushort_as_half((unsigned short)(sc >> 16));
+            const __half2 sA = __halves2half2(s_lo, s_lo), sB = __halves2half2(s_hi, s_hi);
+            const uint32_t wds[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+            uint32_t v[32];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+              uint32_t o[4];
+              q8_to_h4(wds[t], t < 4 ? sA : sB, o);
+#pragma unroll
+              for (int c = 0; c < 4; ++c) v[t * 4 + c] = o[c];
+            }
+            tmem_st32(acol + mat * 64, v);
           }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&C.afull[b]);
         }
-        tmem_st32(acol + mat * 64, v);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&C.afull[b]);
-        mbar_arrive(&C.empty[s]);
+        if (!fine) break;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&C.empty[s]);
       }
       const bool last = (u + 1 == sp.u1) || ((u + 1) % SK == 0);
       if (!last) continue;
@@ -619,14 +629,14 @@ __global__ void __launch_bounds__(kThreads, 1) ts_gemm_kernel(const TsArgs a) {
       if (lane == 0) mbar_arrive(&C.accfree[pb]);
 
       const bool whole = (piece_u0 % SK == 0) && ((u + 1) % SK == 0);
-      if (!whole && !stream_k_finish<S::NMAT * 16>(v, a.part, a.ctr, (int)tile, SK, W, Gs, cta, sp.u0, w, lane, C,
-                                                   wphase, abort_flag, a.status, &ok))
+      if (!whole && !stream_k_finish<S::NMAT * 16>(v, a.part, a.ctr, (int)j_tile, SK, W, Gs, cta, sp.u0, w, lane,
+                                                   C, wphase, abort_flag, a.status, &ok))
         continue;
 
       // ---------------------------------------------------------- finish the tile
-      const int row = (int)(tile * kM) + m;  // r index (pred_h), neuron (pred_s), union position (ffn_up)
+      const int row = tile_of(j_tile) * kM + m;  // r index (pred_h) or neuron (pred_s, ffn_up)
       if constexpr (KIND == K_P1) {
-        if (row < nrows) {
+        if (row < a.nrows) {
           const size_t boff = (size_t)(row >> 4) * kBlk;
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
@@ -639,9 +649,9 @@ __global__ void __launch_bounds__(kThreads, 1) ts_gemm_kernel(const TsArgs a) {
           }
         }
       } else if constexpr (KIND == K_P2) {
-        const bool valid = row < nrows;
+        const bool valid = row < a.nrows;
         const float bias = valid ? __ldg(a.bias + row) : 0.f;
-        const int word = (int)(tile * kM + q * 32) >> 5;
+        const int word = (int)(j_tile * kM + q * 32) >> 5;
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const int n = h * 16 + j;
@@ -649,17 +659,18 @@ __global__ void __launch_bounds__(kThreads, 1) ts_gemm_kernel(const TsArgs a) {
           if (lane == 0 && n < a.B && word < a.nwords) a.mask_out[(size_t)n * a.nwords + word] = bits;
         }
       } else {
-        const bool valid = row < nrows;
-        const int neuron = valid ? __ldg(a.rowlist + row) : 0;
-        const float b1 = (ACT == ACT_RELU && valid) ? __ldg(a.bias + neuron) : 0.f;
-        const size_t boff = (size_t)(row >> 4) * kBlk;
+        // a image position: listed tile j_tile, row m
+        const bool valid = row < a.nrows;
+        const float b1 = (ACT == ACT_RELU && valid) ? __ldg(a.bias + row) : 0.f;
+        const long long pos = j_tile * kM + m;
+        const size_t boff = (size_t)(pos >> 4) * kBlk;
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const int n = h * 16 + j;
           float av = 0.f;
           if (valid && n < a.B) {
-            const uint32_t bits = __ldg(a.mask + (size_t)n * a.nwords + (neuron >> 5));
-            if ((bits >> (neuron & 31)) & 1u) {
+            const uint32_t bits = __ldg(a.mask + (size_t)n * a.nwords + (row >> 5));
+            if ((bits >> (row & 31)) & 1u) {
               if constexpr (ACT == ACT_RELU) {
                 const float pre = v[j] + b1;
                 av = pre > 0.f ? pre : 0.f;
@@ -668,23 +679,22 @@ __global__ void __launch_bounds__(kThreads, 1) ts_gemm_kernel(const TsArgs a) {
               }
             }
           }
-          *reinterpret_cast<__half *>(a.out0 + boff + img_off(n, row & 15)) = __float2half_rn(av);
+          *reinterpret_cast<__half *>(a.out0 + boff + img_off(n, (int)(pos & 15))) = __float2half_rn(av);
         }
       }
     }
   }
-  teardown(C, sp, warp, lane, tmem, S::TMEM_COLS, abort_flag, a.status);
+  teardown(warp, tmem, S::TMEM_COLS);
 }
 
 // ---------------------------------------------------------------- down projection (A in shared memory)
 struct DownArgs {
-  const void *w;                 // W2T rows [f x d] fp16, or packed int4 [f x d/2]
-  const __half *s;               // int4 scales [f x d/32]
-  const int32_t *rowlist;        // union position -> neuron
-  const int32_t *rowcount;       // U
-  int d, B;
-  const unsigned char *aimg;     // a image (union positions as K)
-  float *y;                      // [B x d]
+  CUtensorMap tm;               // W2T: fp16 [f x d] (box 64 x 64) or packed int4 bytes [f x d/2] (box 128 x 64)
+  CUtensorMap ts;               // int4 scale bytes [f x d/16] (box 16 x 64)
+  const uint32_t *uwords;       // union mask words (the same tile list as ffn_up)
+  int nwords, f, d, B;
+  const unsigned char *aimg;    // a image, K = the listed tiles' neurons
+  float *y;                     // [B x d]
   int accumulate;
   float *part;
   int *ctr;
@@ -694,32 +704,35 @@ struct DownArgs {
 template <int WT>
 struct DownShape {
   static constexpr bool Q4 = WT == W_INT4;
-  // staging row pitch per union position: int4 128 B packed + 16 B scales; fp16 512 B + 16 pad
-  static constexpr int ROWB = Q4 ? 144 : 528;
-  static constexpr int SLOTB = kDownStepK * ROWB;
+  // fp16: four 64-column boxes of 64 neurons x 128 B (swizzled, the MMA's
+  // MN-major A as is); int4: one 64 x 128 B packed box + a 64 x 16 B scale box
+  static constexpr int ABYTES = Q4 ? 8192 : 4 * 8192;
+  static constexpr int SBYTES = Q4 ? 1024 : 0;
   static constexpr int IMGB = (kDownStepK / 16) * kBlk;  // 4 KB
-  static constexpr int ABUF = kDownStepK * kDownTileD * 2;  // 32 KB canonical A per step
-  static constexpr int NSLOT_FIT = (kSmemBudget - 2 * ABUF) / (SLOTB + IMGB);
+  static constexpr int IMG_OFF = ABYTES + SBYTES;
+  static constexpr int SLOTB = (IMG_OFF + IMGB + 1023) / 1024 * 1024;
+  static constexpr int ABUF = Q4 ? kDownStepK * kDownTileD * 2 : 0;  // int4: dequantised canonical A, 32 KB
+  static constexpr int NSLOT_FIT = (kSmemBudget - 2 * ABUF) / SLOTB;
   static constexpr int NSLOT = NSLOT_FIT > 6 ? 6 : NSLOT_FIT;
-  static constexpr int A_OFF = 0;
-  static constexpr int IMG_OFF = 2 * ABUF;
-  static constexpr int STAGE_OFF = IMG_OFF + NSLOT * IMGB;
-  static constexpr int CTRL_OFF = STAGE_OFF + NSLOT * SLOTB;
-  static constexpr int SMEM = CTRL_OFF + kCtrlBytes;
+  static constexpr int TX = IMG_OFF + IMGB;
+  static constexpr int A_OFF = NSLOT * SLOTB;
+  static constexpr int CTRL_OFF = A_OFF + 2 * ABUF;
+  static constexpr int SMEM = CTRL_OFF + kCtrlBytes + 1024;
   static constexpr uint32_t TMEM_COLS = 128;  // 2 buffers x 2 M-halves x 32 tokens
   static_assert(NSLOT >= 2, "ring too shallow");
   static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
 template <int WT>
-__global__ void __launch_bounds__(kThreads, 1) ffn_down_kernel(const DownArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) ffn_down_kernel(const __grid_constant__ DownArgs a) {
   using S = DownShape<WT>;
-  extern __shared__ __align__(1024) unsigned char smem[];
-  TsCtrl &C = *reinterpret_cast<TsCtrl *>(smem + S::CTRL_OFF);
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  TcCtrl &C = *reinterpret_cast<TcCtrl *>(smem + S::CTRL_OFF);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, cta = blockIdx.x;
 
-  if (tid == 0) ctrl_init<S::NSLOT>(C);
+  if (tid == 0) ctrl_init<S::NSLOT>(C, S::Q4 ? 9u : 1u);
   if (warp == 1) tmem_alloc(&C.tmem, S::TMEM_COLS);
   tc_fence_before();
   __syncthreads();
@@ -730,13 +743,13 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_down_kernel(const DownArgs a)
   pdl_wait();
   pdl_launch_dependents();
 
-  const int U = *a.rowcount;
+  list_tiles(C, a.uwords, a.nwords, (a.f + kM - 1) / kM);
   const int d = a.d;
   const long long T = (d + kDownTileD - 1) / kDownTileD;
-  const long long SK = (U + kDownStepK - 1) / kDownStepK;
+  const long long SK = (long long)C.n_tiles * (kM / kDownStepK);
   const long long W = T * SK;
   if (W == 0 && !a.accumulate) {
-    // empty union: y = 0
+    // no predicted neuron: y = 0
     const int n = a.B * d;
     for (int e = cta * kThreads + tid; e < n; e += G * kThreads) a.y[e] = 0.f;
   }
@@ -744,63 +757,31 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_down_kernel(const DownArgs a)
   const Span sp = cta < Gs ? span_of(W, Gs, cta) : Span{0, 0};
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    const size_t rowB = S::Q4 ? (size_t)d / 2 : (size_t)d * 2;
-    const size_t srowB = (size_t)d / 16;
-    const unsigned char *wb = reinterpret_cast<const unsigned char *>(a.w);
-    long long i = 0;
-    for (long long u = sp.u0; u < sp.u1; ++u, ++i) {
-      const int s = (int)(i % S::NSLOT);
-      const unsigned ph = (unsigned)((i / S::NSLOT) & 1);
-      if (i >= S::NSLOT) {
-        if (!mbar_wait_warp(&C.empty[s], ph ^ 1u, abort_flag, a.status)) break;
-        if (!mbar_wait_warp(&C.img_empty[s], ph ^ 1u, abort_flag, a.status)) break;
-      }
-      const long long tile = u / SK, step = u % SK;
-      const int dcol0 = (int)tile * kDownTileD;
-      __syncwarp();
+    // ------------------------------------------------------------ producer (one lane)
+    if (lane == 0) {
+      long long i = 0;
+      for (long long u = sp.u0; u < sp.u1; ++u, ++i) {
+        const int s = (int)(i % S::NSLOT);
+        const unsigned ph = (unsigned)((i / S::NSLOT) & 1);
+        if (i >= S::NSLOT && !mbar_wait(&C.empty[s], ph ^ 1u, abort_flag, a.status)) break;
+        const int dcol0 = (int)(u / SK) * kDownTileD;
+        const long long kstep = u % SK;  // 64-neuron half of listed tile kstep / 2
+        const int row0 = C.tlist[kstep >> 1] * kM + (int)(kstep & 1) * kDownStepK;
+        unsigned char *slot = smem + s * S::SLOTB;
+        mbar_expect_tx(&C.full[s], S::TX);
+        if constexpr (S::Q4) {
+          tma_load_2d(su32(slot), &a.tm, dcol0 / 2, row0, &C.full[s]);
+          tma_load_2d(su32(slot + S::ABYTES), &a.ts, dcol0 / 16, row0, &C.full[s]);
+        } else {
 #pragma unroll
-      for (int j = 0; j < kDownStepK / 32; ++j) {
-        const long long p = step * kDownStepK + lane + 32 * j;
-        C.rows[lane + 32 * j] = p < U ? __ldg(a.rowlist + p) : -1;
-      }
-      __syncwarp();
-      if (lane == 0) {
-        mbar_expect_tx(&C.img_full[s], S::IMGB);
-        bulk_g2s(su32(smem + S::IMG_OFF + s * S::IMGB), a.aimg + (size_t)step * S::IMGB, S::IMGB, &C.img_full[s]);
-      }
-      const uint32_t st0 = su32(smem + S::STAGE_OFF + s * S::SLOTB);
-      if constexpr (S::Q4) {
-        const unsigned char *sb = reinterpret_cast<const unsigned char *>(a.s);
-        // 9 pieces per position: 8 x 16 B packed (256 d) + 16 B of the 8 group scales
-#pragma unroll 2
-        for (int qq = lane; qq < kDownStepK * 9; qq += 32) {
-          const int k = qq / 9, c = qq - k * 9;
-          const int rid = C.rows[k];
-          const uint32_t dst = st0 + k * S::ROWB + c * 16;
-          if (c < 8) {
-            const bool ok = rid >= 0 && dcol0 + c * 32 < d;
-            cp16(dst, wb + (ok ? (size_t)rid * rowB + (size_t)dcol0 / 2 + c * 16 : 0), ok ? 16u : 0u);
-          } else {
-            const bool ok = rid >= 0;
-            cp16(dst, sb + (ok ? (size_t)rid * srowB + (size_t)dcol0 / 16 : 0), ok ? 16u : 0u);
-          }
+          for (int mb = 0; mb < 4; ++mb) tma_load_2d(su32(slot + mb * 8192), &a.tm, dcol0 + mb * 64, row0, &C.full[s]);
         }
-      } else {
-#pragma unroll 4
-        for (int qq = lane; qq < kDownStepK * 32; qq += 32) {
-          const int k = qq >> 5, c = qq & 31;
-          const int rid = C.rows[k];
-          const bool ok = rid >= 0 && dcol0 + c * 8 < d;
-          cp16(st0 + k * S::ROWB + c * 16, wb + (ok ? (size_t)rid * rowB + (size_t)(dcol0 + c * 8) * 2 : 0),
-               ok ? 16u : 0u);
-        }
+        bulk_g2s(su32(slot + S::IMG_OFF), a.aimg + (size_t)kstep * S::IMGB, S::IMGB, &C.full[s]);
       }
-      cp_arrive(&C.full[s]);
     }
-    cp_wait_all();
+    __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ MMA issuer (one lane)
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f16(kM, kN, 1, 0);
       long long i = 0;
@@ -809,7 +790,6 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_down_kernel(const DownArgs a)
         const int s = (int)(i % S::NSLOT);
         const unsigned ph = (unsigned)((i / S::NSLOT) & 1);
         const int b = (int)(i & 1);
-        const unsigned bph = (unsigned)((i >> 1) & 1);
         const bool first = (u == sp.u0) || (u % SK == 0);
         if (first) {
           ++piece;
@@ -817,24 +797,30 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_down_kernel(const DownArgs a)
               !mbar_wait(&C.accfree[piece & 1], (unsigned)(((piece >> 1) & 1) ^ 1), abort_flag, a.status))
             break;
         }
-        if (!mbar_wait(&C.afull[b], bph, abort_flag, a.status)) break;
-        if (!mbar_wait(&C.img_full[s], ph, abort_flag, a.status)) break;
+        if (!mbar_wait(&C.full[s], ph, abort_flag, a.status)) break;
+        if (S::Q4 && !mbar_wait(&C.afull[b], (unsigned)((i >> 1) & 1), abort_flag, a.status)) break;
         tc_fence_after();
         const uint32_t acc = tmem + (uint32_t)((piece & 1) * 64);
-        const uint32_t abase = su32(smem + S::A_OFF + b * S::ABUF);
-        const uint32_t img = su32(smem + S::IMG_OFF + s * S::IMGB);
+        const uint32_t slot = su32(smem + s * S::SLOTB);
+        const uint32_t abuf = su32(smem + S::A_OFF + b * S::ABUF);
 #pragma unroll
         for (int j = 0; j < kDownStepK / 16; ++j) {
-          const uint64_t bd = sdesc(img + j * kBlk, 128, 256);
+          const uint64_t bd = sdesc(slot + S::IMG_OFF + j * kBlk, 128, 256);
 #pragma unroll
           for (int hm = 0; hm < 2; ++hm) {
-            // MN-major A: 8-position groups of d 128 B apart, 8-deep K groups 4096 B apart
-            const uint64_t ad = sdesc(abase + (uint32_t)(j * 2 * 4096 + hm * 2048), 4096, 128);
+            uint64_t ad;
+            if constexpr (S::Q4) {
+              // canonical no-swizzle MN-major: 8-position groups of d 128 B apart, 8-neuron groups 4096 B apart
+              ad = sdesc(abuf + (uint32_t)(j * 2 * 4096 + hm * 2048), 4096, 128);
+            } else {
+              // swizzled boxes: 64-column blocks 8 KB apart, 8-neuron groups 1 KB apart
+              ad = sdesc(slot + (uint32_t)(hm * 2 * 8192 + j * 2048), 8192, 1024, kSw128);
+            }
             mma_ss(acc + hm * kN, ad, bd, idesc, (first && j == 0) ? 0u : 1u);
           }
         }
-        mma_commit(&C.afree[b]);
-        mma_commit(&C.img_empty[s]);
+        if (S::Q4) mma_commit(&C.afree[b]);
+        mma_commit(&C.empty[s]);
         const bool last = (u + 1 == sp.u1) || ((u + 1) % SK == 0);
         if (last) mma_commit(&C.accfull[piece & 1]);
       }
@@ -851,30 +837,28 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_down_kernel(const DownArgs a)
     int piece = -1;
     long long piece_u0 = sp.u0;
     for (long long u = sp.u0; u < sp.u1 && ok; ++u, ++i) {
-      const int s = (int)(i % S::NSLOT);
-      const unsigned ph = (unsigned)((i / S::NSLOT) & 1);
-      const int b = (int)(i & 1);
-      const unsigned bph = (unsigned)((i >> 1) & 1);
-      const long long tile = u / SK, step = u % SK;
-      if ((u == sp.u0) || (step == 0)) {
+      const long long tile = u / SK;
+      if ((u == sp.u0) || (u % SK == 0)) {
         ++piece;
         piece_u0 = u;
       }
-      if (!mbar_wait_warp(&C.full[s], ph, abort_flag, a.status)) break;
-      if (i >= 2 && !mbar_wait_warp(&C.afree[b], bph ^ 1u, abort_flag, a.status)) break;
-      const unsigned char *st = smem + S::STAGE_OFF + s * S::SLOTB;
-      unsigned char *ab = smem + S::A_OFF + b * S::ABUF;
-      // canonical MN-major A: (d position m, union position k) at
-      // (k/8)*4096 + (m/8)*128 + (k%8)*16 + (m%8)*2.  A warp's 32 items take
-      // 8 consecutive k (the low bits of the item) so its 16-byte stores and
-      // loads spread over all banks.
       if constexpr (S::Q4) {
+        const int s = (int)(i % S::NSLOT);
+        const unsigned ph = (unsigned)((i / S::NSLOT) & 1);
+        const int b = (int)(i & 1);
+        if (!mbar_wait_warp(&C.full[s], ph, abort_flag, a.status)) break;
+        if (i >= 2 && !mbar_wait_warp(&C.afree[b], (unsigned)(((i >> 1) & 1) ^ 1), abort_flag, a.status)) break;
+        const unsigned char *slot = smem + s * S::SLOTB;
+        unsigned char *ab = smem + S::A_OFF + b * S::ABUF;
+        // item (neuron k, group g of 32 d): packed chunk g of row k sits at (g ^ (k % 8)) * 16 in the
+        // swizzled box; canonical MN-major A element (d m, neuron k) at
+        // (k/8)*4096 + (m/8)*128 + (k%8)*16 + (m%8)*2.  A warp's 32 items take 8
+        // consecutive k so its 16-byte stores spread over all banks.
 #pragma unroll
         for (int it = wt; it < kDownStepK * 8; it += kWorkerThreads) {
           const int k = ((it >> 6) << 3) | (it & 7), g = (it >> 3) & 7;
-          const unsigned char *row = st + k * S::ROWB;
-          const uint4 pk = *reinterpret_cast<const uint4 *>(row + g * 16);
-          const __half sc = *reinterpret_cast<const __half *>(row + 128 + g * 2);
+          const uint4 pk = *reinterpret_cast<const uint4 *>(slot + k * 128 + ((g ^ (k & 7)) << 4));
+          const __half sc = *reinterpret_cast<const __half *>(slot + S::ABYTES + k * 16 + g * 2);
           const __half2 s2 = __halves2half2(sc, sc);
           const uint32_t wds[4] = {pk.x, pk.y, pk.z, pk.w};
           unsigned char *dst = ab + (k >> 3) * 4096 + (k & 7) * 16 + g * 4 * 128;
@@ -885,19 +869,12 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_down_kernel(const DownArgs a)
             *reinterpret_cast<uint4 *>(dst + t * 128) = make_uint4(o[0], o[1], o[2], o[3]);
           }
         }
-      } else {
-#pragma unroll 4
-        for (int it = wt; it < kDownStepK * 32; it += kWorkerThreads) {
-          const int k = ((it >> 8) << 3) | (it & 7), c = (it >> 3) & 31;
-          const uint4 p = *reinterpret_cast<const uint4 *>(st + k * S::ROWB + c * 16);
-          *reinterpret_cast<uint4 *>(ab + (k >> 3) * 4096 + c * 128 + (k & 7) * 16) = p;
+        proxy_fence_async();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&C.afull[b]);
+          mbar_arrive(&C.empty[s]);
         }
-      }
-      proxy_fence_async();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&C.afull[b]);
-        mbar_arrive(&C.empty[s]);
       }
       const bool last = (u + 1 == sp.u1) || ((u + 1) % SK == 0);
       if (!last) continue;
@@ -927,14 +904,17 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_down_kernel(const DownArgs a)
         continue;
       const int dpos = (int)tile * kDownTileD + hm * kM + q * 32 + lane;
       if (dpos < d) {
-        for (int n = 0; n < a.B; ++n) {
-          float *yp = a.y + (size_t)n * d + dpos;
-          *yp = a.accumulate ? *yp + v[n] : v[n];
+#pragma unroll
+        for (int n = 0; n < kN; ++n) {
+          if (n < a.B) {
+            float *yp = a.y + (size_t)n * d + dpos;
+            *yp = a.accumulate ? *yp + v[n] : v[n];
+          }
         }
       }
     }
   }
-  teardown(C, sp, warp, lane, tmem, S::TMEM_COLS, abort_flag, a.status);
+  teardown(warp, tmem, S::TMEM_COLS);
 }
 
 }  // namespace tc

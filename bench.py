@@ -40,9 +40,15 @@ from activation_sparse_decode_gemv_b200 import inputs
 
 def kernels_per_step(cfg, B):
     """Launches of the library's kernels per decode step: batch 1 with fp16 /
-    int4 weights runs as one persistent fused kernel; otherwise five kernels
+    int4 weights runs as one persistent fused kernel; batches 16..32 with fp16
+    / int4 weights run six (token image, two tensor-core predictor GEMMs,
+    compaction, tensor-core up/gate and down GEMMs); otherwise five kernels
     (predictor stage 1, stage 2, compaction, gather, reduction)."""
-    return 1 if (B == 1 and cfg.wtype != "f32" and cfg.r <= 1024 and cfg.d <= 8192) else 5
+    if B == 1 and cfg.wtype != "f32" and cfg.r <= 1024 and cfg.d <= 8192:
+        return 1
+    if 16 <= B <= 32 and cfg.wtype != "f32" and (cfg.wtype != "int4g32" or cfg.d % 256 == 0):
+        return 6
+    return 5
 
 
 def parse(argv=None):
