@@ -74,7 +74,7 @@ WsLayout ws_layout(int dmax, int fmax, int rmax, int B, int G) {
 // counters keep their place whatever batch earlier calls used (they must stay
 // zero between calls; the kernels restore them).
 struct TcLayout {
-  size_t uimg, himg_hi, himg_lo, aimg, part, ctr_p1, ctr_p2, ctr_up, ctr_down, total;
+  size_t uimg, uimg_perm, himg_hi, himg_lo, aimg, part, ctr_p1, ctr_p2, ctr_up, ctr_down, total;
 };
 
 TcLayout tc_layout(int dmax, int fmax, int rmax, int G) {
@@ -82,6 +82,8 @@ TcLayout tc_layout(int dmax, int fmax, int rmax, int G) {
   size_t o = 0;
   const size_t step_img = (size_t)pi::tc::kImgStep / 16 * pi::tc::kBlk;
   L.uimg = o;
+  o = align_up(o + (size_t)((dmax + 127) / 128) * step_img, 256);
+  L.uimg_perm = o;
   o = align_up(o + (size_t)((dmax + 127) / 128) * step_img, 256);
   L.himg_hi = o;
   o = align_up(o + (size_t)((rmax + 127) / 128) * step_img, 256);
@@ -182,6 +184,7 @@ struct Ws {
   int32_t *ulist() const { return reinterpret_cast<int32_t *>(base + L.ulist); }
   float *partial() const { return reinterpret_cast<float *>(base + L.partial); }
   unsigned char *uimg() const { return reinterpret_cast<unsigned char *>(tc + T.uimg); }
+  unsigned char *uimg_perm() const { return reinterpret_cast<unsigned char *>(tc + T.uimg_perm); }
   unsigned char *himg_hi() const { return reinterpret_cast<unsigned char *>(tc + T.himg_hi); }
   unsigned char *himg_lo() const { return reinterpret_cast<unsigned char *>(tc + T.himg_lo); }
   unsigned char *aimg() const { return reinterpret_cast<unsigned char *>(tc + T.aimg); }
@@ -427,7 +430,8 @@ bool tc_ok(const pi_ffn *h, int B) {
 }
 
 template <typename KArg>
-cudaError_t launch_smem(void (*kern)(KArg), int G, int smem, bool *attr_done, cudaStream_t st, const KArg &arg) {
+cudaError_t launch_smem(void (*kern)(KArg), int G, int threads, int smem, bool *attr_done, cudaStream_t st,
+                        const KArg &arg) {
   if (!*attr_done) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
@@ -435,7 +439,7 @@ cudaError_t launch_smem(void (*kern)(KArg), int G, int smem, bool *attr_done, cu
   }
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(G);
-  cfg.blockDim = dim3(TC::kThreads);
+  cfg.blockDim = dim3(threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute at[1];
@@ -449,19 +453,23 @@ cudaError_t launch_smem(void (*kern)(KArg), int G, int smem, bool *attr_done, cu
 template <int KIND, int WT, int ACT>
 cudaError_t ts_launch(const TC::RowArgs &a, int G, cudaStream_t st) {
   static bool attr = false;
-  return launch_smem(TC::row_gemm_kernel<KIND, WT, ACT>, G, TC::RowShape<KIND, WT, ACT>::SMEM, &attr, st, a);
+  using Sh = TC::RowShape<KIND, WT, ACT>;
+  return launch_smem(TC::row_gemm_kernel<KIND, WT, ACT>, G, Sh::THREADS, Sh::SMEM, &attr, st, a);
 }
 
 template <int WT>
 cudaError_t down_launch(const TC::DownArgs &a, int G, cudaStream_t st) {
   static bool attr = false;
-  return launch_smem(TC::ffn_down_kernel<WT>, G, TC::DownShape<WT>::SMEM, &attr, st, a);
+  return launch_smem(TC::ffn_down_kernel<WT>, G, TC::kThreads, TC::DownShape<WT>::SMEM, &attr, st, a);
 }
 
+// token images of u: natural order (predictor, fp16 weights) and, for int4
+// weights, the paired order of the int4 up/gate dequantisation
 cudaError_t tc_u_image(const pi_ffn *h, const void *u, int B, const Ws &w, cudaStream_t st) {
   const int d = h->d.d_model;
   const int total = TC::kN * ((d + 127) / 128) * 16;
-  return launch(TC::u_image_kernel, dim3(cdiv(total, 256)), dim3(256), st, (const __half *)u, B, d, w.uimg());
+  unsigned char *perm = h->d.wtype == PI_W_INT4G32 ? w.uimg_perm() : nullptr;
+  return launch(TC::u_image_kernel, dim3(cdiv(total, 256)), dim3(256), st, (const __half *)u, B, d, w.uimg(), perm);
 }
 
 // steps 1-2 on tensor cores: u image, h = P1 u (hi/lo images), mask words, compaction
@@ -515,7 +523,7 @@ pi_status run_ffn_tc(const pi_ffn *h, const void *u, int B, float *out, int accu
   a.uwords = w.uwords();
   a.nrows = D.d_ffn;
   a.K = D.d_model;
-  a.img0 = w.uimg();
+  a.img0 = D.wtype == PI_W_INT4G32 ? w.uimg_perm() : w.uimg();
   a.bias = D.b_up;
   a.mask = w.mask();
   a.nwords = h->nwords;

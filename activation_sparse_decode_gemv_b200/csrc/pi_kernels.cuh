@@ -212,7 +212,14 @@ __global__ void __launch_bounds__(1024)
       if (!is_union) {
         word = mask[(size_t)b * nwords + w];
       } else {
-        for (int t = 0; t < B; ++t) word |= mask[(size_t)t * nwords + w];
+        // 8 independent loads in flight per round
+        for (int t0 = 0; t0 < B; t0 += 8) {
+          uint32_t v[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) v[k] = t0 + k < B ? mask[(size_t)(t0 + k) * nwords + w] : 0u;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) word |= v[k];
+        }
         uwords[w] = word;
       }
     }

@@ -47,8 +47,9 @@ namespace tc {
 constexpr int kN = 32;        // MMA N: token columns (batches of 16..32 are zero-padded)
 constexpr int kM = 128;       // MMA M: rows of a tile
 constexpr int kBlk = 1024;    // bytes of one 16-deep K block of a token image
-constexpr int kThreads = 320; // warp 0 producer, warp 1 MMA issuer, warps 2..9 workers
-constexpr int kWorkerThreads = 256;
+// warp 0 producer, warp 1 MMA issuer, warps 2.. workers (8, or 16 for int4 dequant)
+constexpr int kThreads = 320;      // 8 worker warps
+constexpr int kMaxThreads = 576;   // 16 worker warps
 constexpr int kSmemBudget = 216 * 1024;
 constexpr int kPartFloats = 128 * 64;  // largest per-piece partial (floats)
 constexpr int kDownTileD = 256;        // d positions per down-projection tile (two M=128 MMAs)
@@ -78,12 +79,24 @@ PI_DEV void mbar_expect_tx(uint64_t *b, unsigned bytes) {
   asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(su32(b)), "r"(bytes)
                : "memory");
 }
+// non-blocking test of the phase with the given parity
 PI_DEV bool mbar_test(uint64_t *b, unsigned parity) {
   uint32_t ok;
   asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(ok)
       : "r"(su32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// try_wait with a suspend-time hint: the thread is parked until the phase
+// completes or the hint elapses, instead of spinning on the barrier
+PI_DEV bool mbar_try(uint64_t *b, unsigned parity, unsigned hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(su32(b)), "r"(parity), "r"(hint_ns)
       : "memory");
   return ok != 0;
 }
@@ -92,7 +105,7 @@ PI_DEV bool mbar_test(uint64_t *b, unsigned parity) {
 __device__ __noinline__ bool mbar_wait_slow(uint64_t *b, unsigned parity, volatile int *abort_flag, int *status) {
   const unsigned long long t0 = now_ns();
   for (;;) {
-    if (mbar_test(b, parity)) return true;
+    if (mbar_try(b, parity, 20000u)) return true;
     if (*abort_flag) return false;
     if (now_ns() - t0 > kWaitNs) {
       set_status(status, kStatusTimeout);
@@ -203,6 +216,25 @@ PI_DEV void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
 }
 
+PI_DEV void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr)
+               : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int j = 0; j < 8; ++j) v[j] = __uint_as_float(r[j]);
+}
+PI_DEV void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
 // byte offset of (token n, k) inside one 16-deep K block of a token image
 PI_DEV uint32_t img_off(int n, int k) {
   return (uint32_t)((n >> 3) * 256 + (k >> 3) * 128 + (n & 7) * 16 + (k & 7) * 2);
@@ -229,6 +261,21 @@ PI_DEV void q8_to_h4(uint32_t w, __half2 s2, uint32_t (&o)[4]) {
   }
 }
 
+// One 32-bit word of packed nibbles n0..n7 to the four fp16 pairs
+// (n0, n4), (n1, n5), (n2, n6), (n3, n7), each s * (q - 8).  Pairing nibble j
+// with nibble j + 4 needs only a shift and a masked OR per pair; the K order
+// this gives (positions 2j, 2j+1 of an 8-block hold elements j, j+4) is
+// matched by the permuted token image (u_image_kernel).
+PI_DEV void q8_to_h4_paired(uint32_t w, __half2 s2, uint32_t (&o)[4]) {
+  const __half2 off = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t p = ((w >> (4 * j)) & 0x000F000Fu) | 0x64006400u;
+    __half2 v = __hmul2(__hsub2(*reinterpret_cast<const __half2 *>(&p), off), s2);
+    o[j] = *reinterpret_cast<uint32_t *>(&v);
+  }
+}
+
 // ---------------------------------------------------------------- stream-K
 struct Span {
   long long u0, u1;  // this CTA's units [u0, u1)
@@ -238,9 +285,12 @@ PI_DEV Span span_of(long long W, int G, int c) { return Span{W * c / G, W * (c +
 PI_DEV int owner_of(long long u, long long W, int G) { return (int)(((u + 1) * G + W - 1) / W) - 1; }
 
 // ---------------------------------------------------------------- token image
-// u [B x d] fp16 -> image of ceil(d/128)*8 blocks; tokens >= B and k >= d are 0
+// u [B x d] fp16 -> image of ceil(d/128)*8 blocks; tokens >= B and k >= d are
+// 0.  img_perm (optional) receives the same image with every 8-element K
+// block in the order 0 4 1 5 2 6 3 7 (the order of q8_to_h4_paired).
 __global__ void __launch_bounds__(256) u_image_kernel(const __half *__restrict__ u, int B, int d,
-                                                      unsigned char *__restrict__ img) {
+                                                      unsigned char *__restrict__ img,
+                                                      unsigned char *__restrict__ img_perm) {
   pdl_wait();
   pdl_launch_dependents();
   const int nblk = (d + kImgStep - 1) / kImgStep * 8;
@@ -253,6 +303,10 @@ __global__ void __launch_bounds__(256) u_image_kernel(const __half *__restrict__
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (n < B && k0 < d) v = *reinterpret_cast<const uint4 *>(u + (size_t)n * d + k0);
     *reinterpret_cast<uint4 *>(img + (size_t)blk * kBlk + img_off(n, kh * 8)) = v;
+    if (img_perm)
+      *reinterpret_cast<uint4 *>(img_perm + (size_t)blk * kBlk + img_off(n, kh * 8)) =
+          make_uint4(__byte_perm(v.x, v.z, 0x5410), __byte_perm(v.x, v.z, 0x7632), __byte_perm(v.y, v.w, 0x5410),
+                     __byte_perm(v.y, v.w, 0x7632));
   }
 }
 
@@ -265,27 +319,27 @@ struct TcCtrl {
   int abort_flag;
   int is_last;
   int n_tiles;    // tiles listed in tlist
-  int wcnt[kThreads / 32];
+  int wcnt[kMaxThreads / 32];
   int tlist[kMaxTiles];  // ffn kernels: 128-neuron tiles holding a predicted neuron
 };
 constexpr int kCtrlBytes = 5120;
 static_assert(sizeof(TcCtrl) <= kCtrlBytes, "control block");
 
-// empty_count: arrivals that free a ring slot (1: the MMA's commit; 9: the
-// 8 worker warps that read the slot and the MMA's commit)
+// nw: worker warps.  empty_count: arrivals that free a ring slot (1: the
+// MMA's commit; nw + 1: the worker warps that read the slot and the commit)
 template <int NSLOT>
-PI_DEV void ctrl_init(TcCtrl &C, unsigned empty_count) {
+PI_DEV void ctrl_init(TcCtrl &C, unsigned nw, unsigned empty_count) {
   for (int s = 0; s < NSLOT; ++s) {
     mbar_init(&C.full[s], 1);  // the producer's expect_tx; TMA completes the bytes
     mbar_init(&C.empty[s], empty_count);
   }
   for (int b = 0; b < 2; ++b) {
-    mbar_init(&C.afull[b], 8);
+    mbar_init(&C.afull[b], nw);
     mbar_init(&C.afree[b], 1);
     mbar_init(&C.accfull[b], 1);
-    mbar_init(&C.accfree[b], 8);
+    mbar_init(&C.accfree[b], nw);
   }
-  mbar_init(&C.wbar, kWorkerThreads);
+  mbar_init(&C.wbar, nw * 32);
   C.abort_flag = 0;
   C.is_last = 0;
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -294,9 +348,9 @@ PI_DEV void ctrl_init(TcCtrl &C, unsigned empty_count) {
 // All threads: list the 128-neuron tiles that hold a set bit of the union
 // words (4 words per tile), in ascending order, into C.tlist / C.n_tiles.
 PI_DEV void list_tiles(TcCtrl &C, const uint32_t *uwords, int nwords, int n_all) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nthreads = blockDim.x;
   int base = 0;
-  for (int t0 = 0; t0 < n_all; t0 += kThreads) {
+  for (int t0 = 0; t0 < n_all; t0 += nthreads) {
     const int t = t0 + tid;
     bool act = false;
     if (t < n_all) {
@@ -311,7 +365,7 @@ PI_DEV void list_tiles(TcCtrl &C, const uint32_t *uwords, int nwords, int n_all)
     for (int w = 0; w < warp; ++w) off += C.wcnt[w];
     if (act) C.tlist[off + __popc(bal & ((1u << lane) - 1u))] = t;
     int tot = 0;
-    for (int w = 0; w < kThreads / 32; ++w) tot += C.wcnt[w];
+    for (int w = 0; w < nthreads / 32; ++w) tot += C.wcnt[w];
     base += tot;
     __syncthreads();
   }
@@ -352,19 +406,31 @@ PI_DEV bool stream_k_finish(float (&v)[NV], float *part, int *ctr, int tile, lon
     return false;
   }
   if (!C.is_last) return false;
+  // pieces are loaded PB at a time (independent loads in flight) and added in K order
+  constexpr int PB = NV >= 16 ? 2 : 4;
   float acc[NV];
 #pragma unroll
   for (int j = 0; j < NV; ++j) acc[j] = 0.f;
-  for (int c = c0; c <= c1; ++c) {
-    if (c == cta) {
+  for (int c = c0; c <= c1; c += PB) {
+    float t[PB][NV];
 #pragma unroll
-      for (int j = 0; j < NV; ++j) acc[j] += v[j];
-    } else {
-      const int cslot = (int)(span_of(W, G, c).u0 / SK) == tile ? 0 : 1;
-      const float *pp = part + ((size_t)c * 2 + cslot) * kPartFloats;
+    for (int k = 0; k < PB; ++k) {
+      const int cc = c + k;
+      if (cc <= c1 && cc != cta) {
+        const int cslot = (int)(span_of(W, G, cc).u0 / SK) == tile ? 0 : 1;
+        const float *pp = part + ((size_t)cc * 2 + cslot) * kPartFloats;
 #pragma unroll
-      for (int j = 0; j < NV; ++j) acc[j] += __ldcg(pp + (w * NV + j) * 32 + lane);
+        for (int j = 0; j < NV; ++j) t[k][j] = __ldcg(pp + (w * NV + j) * 32 + lane);
+      } else {
+#pragma unroll
+        for (int j = 0; j < NV; ++j) t[k][j] = v[j];
+      }
     }
+#pragma unroll
+    for (int k = 0; k < PB; ++k)
+      if (c + k <= c1)
+#pragma unroll
+        for (int j = 0; j < NV; ++j) acc[j] += t[k][j];
   }
 #pragma unroll
   for (int j = 0; j < NV; ++j) v[j] = acc[j];
@@ -421,13 +487,18 @@ struct RowShape {
   static constexpr int ACC_COLS = NMAT * kN;        // per accumulator buffer
   static constexpr int A_COLS = NMAT * 64;          // int4: per tensor-memory A buffer (128 K)
   static constexpr uint32_t TMEM_COLS = Q4 ? 512 : 128;
+  static constexpr int NW = Q4 ? 16 : 8;            // worker warps
+  static constexpr int THREADS = 64 + 32 * NW;
+  static constexpr int KQ = NW / 4;                 // workers per tensor-memory lane quarter
+  static constexpr int TOKW = kN / KQ;              // epilogue token columns per worker
+  static constexpr int NV = NMAT * TOKW;            // accumulator values per worker thread
   static_assert(NSLOT >= 2, "ring too shallow");
   static_assert(SMEM <= 227 * 1024, "shared memory");
   static_assert(2 * ACC_COLS + (Q4 ? 2 * A_COLS : 0) <= (int)TMEM_COLS, "tensor memory");
 };
 
 template <int KIND, int WT, int ACT>
-__global__ void __launch_bounds__(kThreads, 1) row_gemm_kernel(const __grid_constant__ RowArgs a) {
+__global__ void __launch_bounds__(RowShape<KIND, WT, ACT>::THREADS, 1) row_gemm_kernel(const __grid_constant__ RowArgs a) {
   using S = RowShape<KIND, WT, ACT>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -435,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1) row_gemm_kernel(const __grid_cons
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, cta = blockIdx.x;
 
-  if (tid == 0) ctrl_init<S::NSLOT>(C, S::Q4 ? 9u : 1u);
+  if (tid == 0) ctrl_init<S::NSLOT>(C, S::NW, S::Q4 ? S::NW + 1u : 1u);
   if (warp == 1) tmem_alloc(&C.tmem, S::TMEM_COLS);
   tc_fence_before();
   __syncthreads();
@@ -462,30 +533,33 @@ __global__ void __launch_bounds__(kThreads, 1) row_gemm_kernel(const __grid_cons
   auto tile_of = [&](long long j) -> int { return KIND == K_UP ? C.tlist[j] : (int)j; };
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer (one lane)
-    if (lane == 0) {
-      long long i = 0;
-      for (long long u = sp.u0; u < sp.u1; ++u, ++i) {
-        const int s = (int)(i % S::NSLOT);
-        const unsigned ph = (unsigned)((i / S::NSLOT) & 1);
-        if (i >= S::NSLOT && !mbar_wait(&C.empty[s], ph ^ 1u, abort_flag, a.status)) break;
-        const int row0 = tile_of(u / SK) * kM;
-        const int k0 = (int)(u % SK) * S::STEPK;
-        unsigned char *slot = smem + s * S::SLOTB;
-        mbar_expect_tx(&C.full[s], S::TX);
-#pragma unroll
-        for (int mat = 0; mat < S::NMAT; ++mat) {
-          tma_load_2d(su32(slot + mat * S::ABOX), mat == 0 ? &a.tm0 : &a.tm1, S::Q4 ? k0 / 2 : k0, row0, &C.full[s]);
-          if constexpr (S::Q4)
-            tma_load_2d(su32(slot + S::SC_OFF + mat * S::SBOX), mat == 0 ? &a.ts0 : &a.ts1, k0 / 16, row0, &C.full[s]);
-        }
+    // ------------------------------------------------------------ producer warp
+    // A thread issues its bulk copies one after another, so the copies of a
+    // unit are spread over the lanes: lane c issues copy c.
+    long long i = 0;
+    for (long long u = sp.u0; u < sp.u1; ++u, ++i) {
+      const int s = (int)(i % S::NSLOT);
+      const unsigned ph = (unsigned)((i / S::NSLOT) & 1);
+      if (i >= S::NSLOT && !mbar_wait_warp(&C.empty[s], ph ^ 1u, abort_flag, a.status)) break;
+      const int row0 = tile_of(u / SK) * kM;
+      const int k0 = (int)(u % SK) * S::STEPK;
+      unsigned char *slot = smem + s * S::SLOTB;
+      if (lane == 0) mbar_expect_tx(&C.full[s], S::TX);
+      __syncwarp();
+      // copies: A boxes (lanes 0..NMAT-1), int4 scale boxes (NMAT..2 NMAT-1), images (next lanes)
+      constexpr int LS = S::NMAT, LI = S::Q4 ? 2 * S::NMAT : S::NMAT;
+      if (lane < LS) {
+        tma_load_2d(su32(slot + lane * S::ABOX), lane == 0 ? &a.tm0 : &a.tm1, S::Q4 ? k0 / 2 : k0, row0, &C.full[s]);
+      } else if (S::Q4 && lane < LI) {
+        const int mat = lane - LS;
+        tma_load_2d(su32(slot + S::SC_OFF + mat * S::SBOX), mat == 0 ? &a.ts0 : &a.ts1, k0 / 16, row0, &C.full[s]);
+      } else if (lane < LI + S::NIMG) {
+        const int nb = lane - LI;
         const size_t ib = (size_t)(k0 / 16) * kBlk;
-        bulk_g2s(su32(slot + S::IMG_OFF), a.img0 + ib, (S::STEPK / 16) * kBlk, &C.full[s]);
-        if (S::NIMG == 2)
-          bulk_g2s(su32(slot + S::IMG_OFF + (S::STEPK / 16) * kBlk), a.img1 + ib, (S::STEPK / 16) * kBlk, &C.full[s]);
+        bulk_g2s(su32(slot + S::IMG_OFF + nb * (S::STEPK / 16) * kBlk), (nb == 0 ? a.img0 : a.img1) + ib,
+                 (S::STEPK / 16) * kBlk, &C.full[s]);
       }
     }
-    __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (one lane)
     if (lane == 0) {
@@ -547,9 +621,9 @@ __global__ void __launch_bounds__(kThreads, 1) row_gemm_kernel(const __grid_cons
     __syncwarp();
   } else {
     // ------------------------------------------------------------ workers: int4 A operand + epilogues
-    const int w = warp - 2;       // 0..7
+    const int w = warp - 2;       // 0..NW-1
     const int q = warp & 3;       // tensor-memory lane quarter of this warp
-    const int h = w >> 2;         // K half of a dequant step; token half of the epilogue
+    const int kq = w >> 2;        // slice of a dequant step's K; of the epilogue's tokens
     const int m = q * 32 + lane;  // row within the tile
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
     unsigned wphase = 0;
@@ -577,28 +651,25 @@ __global__ void __launch_bounds__(kThreads, 1) row_gemm_kernel(const __grid_cons
             fine = false;
             break;
           }
-          const uint32_t acol = lane_base + (uint32_t)(2 * S::ACC_COLS + b * S::A_COLS + h * 32);
+          // this thread: row m, the 32-element group g of the unit (one 16-byte chunk)
+          const int g = sub * 4 + kq;
+          const uint32_t acol = lane_base + (uint32_t)(2 * S::ACC_COLS + b * S::A_COLS + kq * 16);
 #pragma unroll
           for (int mat = 0; mat < S::NMAT; ++mat) {
-            // packed row m of the swizzled box: 16-byte chunk c sits at (c ^ (m % 8)) * 16
-            const unsigned char *row = slot + mat * S::ABOX + m * 128;
-            const int c0 = sub * 4 + h * 2;
-            const uint4 p0 = *reinterpret_cast<const uint4 *>(row + ((c0 ^ (m & 7)) << 4));
-            const uint4 p1 = *reinterpret_cast<const uint4 *>(row + (((c0 + 1) ^ (m & 7)) << 4));
-            const uint32_t sc = *reinterpret_cast<const uint32_t *>(slot + S::SC_OFF + mat * S::SBOX + m * 16 + c0 * 2);
-            const __half s_lo = __ushort_as_half((unsigned short)(sc & 0xFFFFu));
-            const __half s_hi = __ushort_as_half((unsigned short)(sc >> 16));
-            const __half2 sA = __halves2half2(s_lo, s_lo), sB = __halves2half2(s_hi, s_hi);
-            const uint32_t wds[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-            uint32_t v[32];
+            // packed row m of the swizzled box: 16-byte chunk g sits at (g ^ (m % 8)) * 16
+            const uint4 pk = *reinterpret_cast<const uint4 *>(slot + mat * S::ABOX + m * 128 + ((g ^ (m & 7)) << 4));
+            const __half sc = *reinterpret_cast<const __half *>(slot + S::SC_OFF + mat * S::SBOX + m * 16 + g * 2);
+            const __half2 s2 = __halves2half2(sc, sc);
+            const uint32_t wds[4] = {pk.x, pk.y, pk.z, pk.w};
+            uint32_t v[16];
 #pragma unroll
-            for (int t = 0; t < 8; ++t) {
+            for (int t = 0; t < 4; ++t) {
               uint32_t o[4];
-              q8_to_h4(wds[t], t < 4 ? sA : sB, o);
+              q8_to_h4_paired(wds[t], s2, o);
 #pragma unroll
               for (int c = 0; c < 4; ++c) v[t * 4 + c] = o[c];
             }
-            tmem_st32(acol + mat * 64, v);
+            tmem_st16(acol + mat * 64, v);
           }
           tmem_wait_st();
           tc_fence_before();
@@ -616,21 +687,29 @@ __global__ void __launch_bounds__(kThreads, 1) row_gemm_kernel(const __grid_cons
       const int pb = piece & 1;
       if (!mbar_wait_warp(&C.accfull[pb], (unsigned)((piece >> 1) & 1), abort_flag, a.status)) break;
       tc_fence_after();
-      float v[S::NMAT * 16];
+      float v[S::NV];
 #pragma unroll
       for (int mat = 0; mat < S::NMAT; ++mat) {
-        float t[16];
-        tmem_ld16(lane_base + (uint32_t)(pb * S::ACC_COLS + mat * kN + h * 16), t);
+        const uint32_t col = lane_base + (uint32_t)(pb * S::ACC_COLS + mat * kN + kq * S::TOKW);
+        if constexpr (S::TOKW == 16) {
+          float t[16];
+          tmem_ld16(col, t);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) v[mat * 16 + j] = t[j];
+          for (int j = 0; j < 16; ++j) v[mat * 16 + j] = t[j];
+        } else {
+          float t[8];
+          tmem_ld8(col, t);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) v[mat * 8 + j] = t[j];
+        }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&C.accfree[pb]);
 
       const bool whole = (piece_u0 % SK == 0) && ((u + 1) % SK == 0);
-      if (!whole && !stream_k_finish<S::NMAT * 16>(v, a.part, a.ctr, (int)j_tile, SK, W, Gs, cta, sp.u0, w, lane,
-                                                   C, wphase, abort_flag, a.status, &ok))
+      if (!whole && !stream_k_finish<S::NV>(v, a.part, a.ctr, (int)j_tile, SK, W, Gs, cta, sp.u0, w, lane, C,
+                                            wphase, abort_flag, a.status, &ok))
         continue;
 
       // ---------------------------------------------------------- finish the tile
@@ -639,8 +718,8 @@ __global__ void __launch_bounds__(kThreads, 1) row_gemm_kernel(const __grid_cons
         if (row < a.nrows) {
           const size_t boff = (size_t)(row >> 4) * kBlk;
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int n = h * 16 + j;
+          for (int j = 0; j < S::TOKW; ++j) {
+            const int n = kq * S::TOKW + j;
             const __half hi = __float2half_rn(v[j]);
             const __half lo = __float2half_rn(v[j] - __half2float(hi));
             const uint32_t o = img_off(n, row & 15);
@@ -653,8 +732,8 @@ __global__ void __launch_bounds__(kThreads, 1) row_gemm_kernel(const __grid_cons
         const float bias = valid ? __ldg(a.bias + row) : 0.f;
         const int word = (int)(j_tile * kM + q * 32) >> 5;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int n = h * 16 + j;
+        for (int j = 0; j < S::TOKW; ++j) {
+          const int n = kq * S::TOKW + j;
           const unsigned bits = __ballot_sync(0xffffffffu, valid && (v[j] + bias > 0.f));
           if (lane == 0 && n < a.B && word < a.nwords) a.mask_out[(size_t)n * a.nwords + word] = bits;
         }
@@ -665,8 +744,8 @@ __global__ void __launch_bounds__(kThreads, 1) row_gemm_kernel(const __grid_cons
         const long long pos = j_tile * kM + m;
         const size_t boff = (size_t)(pos >> 4) * kBlk;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int n = h * 16 + j;
+        for (int j = 0; j < S::TOKW; ++j) {
+          const int n = kq * S::TOKW + j;
           float av = 0.f;
           if (valid && n < a.B) {
             const uint32_t bits = __ldg(a.mask + (size_t)n * a.nwords + (row >> 5));
@@ -675,7 +754,7 @@ __global__ void __launch_bounds__(kThreads, 1) row_gemm_kernel(const __grid_cons
                 const float pre = v[j] + b1;
                 av = pre > 0.f ? pre : 0.f;
               } else {
-                av = silu(v[16 + j]) * v[j];  // silu(gate) * up
+                av = silu(v[S::TOKW + j]) * v[j];  // silu(gate) * up
               }
             }
           }
@@ -732,7 +811,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_down_kernel(const __grid_cons
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, cta = blockIdx.x;
 
-  if (tid == 0) ctrl_init<S::NSLOT>(C, S::Q4 ? 9u : 1u);
+  if (tid == 0) ctrl_init<S::NSLOT>(C, 8u, S::Q4 ? 9u : 1u);
   if (warp == 1) tmem_alloc(&C.tmem, S::TMEM_COLS);
   tc_fence_before();
   __syncthreads();
@@ -757,29 +836,30 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_down_kernel(const __grid_cons
   const Span sp = cta < Gs ? span_of(W, Gs, cta) : Span{0, 0};
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer (one lane)
-    if (lane == 0) {
-      long long i = 0;
-      for (long long u = sp.u0; u < sp.u1; ++u, ++i) {
-        const int s = (int)(i % S::NSLOT);
-        const unsigned ph = (unsigned)((i / S::NSLOT) & 1);
-        if (i >= S::NSLOT && !mbar_wait(&C.empty[s], ph ^ 1u, abort_flag, a.status)) break;
-        const int dcol0 = (int)(u / SK) * kDownTileD;
-        const long long kstep = u % SK;  // 64-neuron half of listed tile kstep / 2
-        const int row0 = C.tlist[kstep >> 1] * kM + (int)(kstep & 1) * kDownStepK;
-        unsigned char *slot = smem + s * S::SLOTB;
-        mbar_expect_tx(&C.full[s], S::TX);
+    // ------------------------------------------------------------ producer warp (lane c issues copy c)
+    long long i = 0;
+    for (long long u = sp.u0; u < sp.u1; ++u, ++i) {
+      const int s = (int)(i % S::NSLOT);
+      const unsigned ph = (unsigned)((i / S::NSLOT) & 1);
+      if (i >= S::NSLOT && !mbar_wait_warp(&C.empty[s], ph ^ 1u, abort_flag, a.status)) break;
+      const int dcol0 = (int)(u / SK) * kDownTileD;
+      const long long kstep = u % SK;  // 64-neuron half of listed tile kstep / 2
+      const int row0 = C.tlist[kstep >> 1] * kM + (int)(kstep & 1) * kDownStepK;
+      unsigned char *slot = smem + s * S::SLOTB;
+      if (lane == 0) mbar_expect_tx(&C.full[s], S::TX);
+      __syncwarp();
+      constexpr int NA = S::Q4 ? 2 : 4;  // int4: packed + scales; fp16: four 64-column boxes
+      if (lane < NA) {
         if constexpr (S::Q4) {
-          tma_load_2d(su32(slot), &a.tm, dcol0 / 2, row0, &C.full[s]);
-          tma_load_2d(su32(slot + S::ABYTES), &a.ts, dcol0 / 16, row0, &C.full[s]);
+          if (lane == 0) tma_load_2d(su32(slot), &a.tm, dcol0 / 2, row0, &C.full[s]);
+          else tma_load_2d(su32(slot + S::ABYTES), &a.ts, dcol0 / 16, row0, &C.full[s]);
         } else {
-#pragma unroll
-          for (int mb = 0; mb < 4; ++mb) tma_load_2d(su32(slot + mb * 8192), &a.tm, dcol0 + mb * 64, row0, &C.full[s]);
+          tma_load_2d(su32(slot + lane * 8192), &a.tm, dcol0 + lane * 64, row0, &C.full[s]);
         }
+      } else if (lane == NA) {
         bulk_g2s(su32(slot + S::IMG_OFF), a.aimg + (size_t)kstep * S::IMGB, S::IMGB, &C.full[s]);
       }
     }
-    __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (one lane)
     if (lane == 0) {
@@ -855,7 +935,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_down_kernel(const __grid_cons
         // (k/8)*4096 + (m/8)*128 + (k%8)*16 + (m%8)*2.  A warp's 32 items take 8
         // consecutive k so its 16-byte stores spread over all banks.
 #pragma unroll
-        for (int it = wt; it < kDownStepK * 8; it += kWorkerThreads) {
+        for (int it = wt; it < kDownStepK * 8; it += kThreads - 64) {
           const int k = ((it >> 6) << 3) | (it & 7), g = (it >> 3) & 7;
           const uint4 pk = *reinterpret_cast<const uint4 *>(slot + k * 128 + ((g ^ (k & 7)) << 4));
           const __half sc = *reinterpret_cast<const __half *>(slot + S::ABYTES + k * 16 + g * 2);
