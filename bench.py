@@ -148,14 +148,17 @@ def step_bytes(cfg: inputs.Config, B: int, n_union: int) -> int:
 
 # ----------------------------------------------------------------------------- profile summaries
 
-def kernel_source_hash() -> str:
-    """Hash of the CUDA sources; a profile summary's counters apply only to the
-    kernels built from the sources it records."""
-    import glob
+# device sources the fused batch-1 kernel is compiled from
+FUSED_SOURCES = ("pi_fused.cuh", "pi_device.cuh")
+
+
+def kernel_source_hash(files=FUSED_SOURCES) -> str:
+    """Hash of the CUDA sources a kernel is built from; a profile summary's
+    counters apply only to the kernel built from the sources it records."""
     import hashlib
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "activation_sparse_decode_gemv_b200", "csrc", "*"))):
-        with open(p, "rb") as fh:
+    for name in files:
+        with open(os.path.join(ROOT, "activation_sparse_decode_gemv_b200", "csrc", name), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
