@@ -24,6 +24,36 @@
 
 namespace pi {
 
+// ============================================================== mixed-precision dots
+// 8 fp16 weights times 8 fp16 inputs (16 B each) into two fp32 chains with
+// the mixed-precision FMA: the product of two fp16 values is exact in fp32,
+// so each step equals fmaf((float)w, (float)u, acc) bit for bit, without the
+// conversions.
+PI_DEV void mdot8(const uint4 &w, const uint4 &u, float &x, float &y) {
+  const unsigned ws[4] = {w.x, w.y, w.z, w.w}, us[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    asm("{\n .reg .b16 al, ah, bl, bh;\n mov.b32 {al, ah}, %2;\n mov.b32 {bl, bh}, %3;\n"
+        " fma.rn.f32.f16 %0, al, bl, %0;\n fma.rn.f32.f16 %1, ah, bh, %1;\n}\n"
+        : "+f"(x), "+f"(y)
+        : "r"(ws[k]), "r"(us[k]));
+}
+// the 8 int4 codes of one 32-bit word (element 2k = low nibble of byte k) as
+// four fp16 pairs (q - 8), in element order: 0x6400 | q is the fp16 value
+// 1024 + q, and subtracting 1032 is exact
+PI_DEV uint4 q8_pairs(uint32_t w) {
+  const __half2 off = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));
+  uint32_t o[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t t = w >> (8 * k);
+    const uint32_t hb = (t & 0xFu) | ((t & 0xF0u) << 12) | 0x64006400u;
+    const __half2 v = __hsub2(*reinterpret_cast<const __half2 *>(&hb), off);
+    o[k] = *reinterpret_cast<const uint32_t *>(&v);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 // ============================================================== rmsnorm
 // u_b = fp16(x_b / sqrt(mean(x_b^2) + 1e-6)).  The sum of squares is taken in
 // double (each square is exact), the mean is rounded once to float, and the
@@ -88,7 +118,15 @@ __global__ void __launch_bounds__(256)
       if (c + 32 * q < nch) {
 #pragma unroll
         for (int t = 0; t < NB; ++t)
-          if (t0 + t < B) acc[t] += chunk_dot<WT>(w[q], ubase + (size_t)t * ub, (c + 32 * q) * E);
+          if (t0 + t < B) {
+            if constexpr (WT == W_F16) {
+              float x = 0.f, y = 0.f;
+              mdot8(w[q], ld_keep16(ubase + (size_t)t * ub + (size_t)(c + 32 * q) * 16), x, y);
+              acc[t] += x + y;
+            } else {
+              acc[t] += chunk_dot<WT>(w[q], ubase + (size_t)t * ub, (c + 32 * q) * E);
+            }
+          }
       }
   }
 #pragma unroll
@@ -314,40 +352,75 @@ PI_DEV int virtual_len(const int32_t *ucount, const int32_t *uprefix, int hot_de
 }
 PI_DEV int chunk_begin(int c, int V, int G) { return (int)(((long long)c * V) / G); }
 
-// one warp: dots of row i with the NB tokens of this group; all lanes get the sums
-template <int NB, int WT>
-PI_DEV void row_dot(const void *W, const __half *S, int i, const void *u, int d, int B, int t0, int lane,
-                    float out[NB]) {
+// one warp: dots of row i of NR matrices (W[0], W[1]: up and gate) with the
+// NB tokens of this group; all lanes get the sums.  fp16 and int4 weights
+// multiply the fp16 tokens with the mixed-precision FMA (no conversions);
+// the rows of both matrices stream in the same loop (8 loads per lane in
+// flight in total).
+template <int NB, int WT, int NR>
+PI_DEV void row_dots(const void *const *W, const __half *const *S, int i, const void *u, int d, int B, int t0,
+                     int lane, float (&out)[NR][NB]) {
   constexpr int E = Chunk<WT>::elems;
-  constexpr int UNR = 8;
+  constexpr int UNR = 8 / NR;  // 8 loads per lane in flight over the NR rows
   const size_t rb = WT == W_F32 ? (size_t)d * 4 : WT == W_F16 ? (size_t)d * 2 : (size_t)d / 2;
   const size_t ub = WT == W_F32 ? (size_t)d * 4 : (size_t)d * 2;
-  const char *row = reinterpret_cast<const char *>(W) + (size_t)i * rb;
   const char *ubase = reinterpret_cast<const char *>(u) + (size_t)t0 * ub;
   const int nch = d / E;
 #pragma unroll
-  for (int t = 0; t < NB; ++t) out[t] = 0.f;
-  for (int c = lane; c < nch; c += 32 * UNR) {
-    uint4 w[UNR];
+  for (int m = 0; m < NR; ++m)
 #pragma unroll
-    for (int q = 0; q < UNR; ++q)
-      if (c + 32 * q < nch) w[q] = ld_stream16(row + (size_t)(c + 32 * q) * 16);
+    for (int t = 0; t < NB; ++t) out[m][t] = 0.f;
+  for (int c = lane; c < nch; c += 32 * UNR) {
+    uint4 w[NR][UNR];
+#pragma unroll
+    for (int m = 0; m < NR; ++m) {
+      const char *row = reinterpret_cast<const char *>(W[m]) + (size_t)i * rb;
+#pragma unroll
+      for (int q = 0; q < UNR; ++q)
+        if (c + 32 * q < nch) w[m][q] = ld_stream16(row + (size_t)(c + 32 * q) * 16);
+    }
 #pragma unroll
     for (int q = 0; q < UNR; ++q) {
       const int cc = c + 32 * q;
-      if (cc < nch) {
-        const float sc = (WT == W_INT4) ? __half2float(S[(size_t)i * (d / 32) + cc]) : 1.0f;
+      if (cc >= nch) continue;
 #pragma unroll
-        for (int t = 0; t < NB; ++t)
-          if (t0 + t < B) {
-            const float p = chunk_dot<WT>(w[q], ubase + (size_t)t * ub, cc * E);
-            out[t] = (WT == W_INT4) ? fmaf(sc, p, out[t]) : out[t] + p;
-          }
+      for (int m = 0; m < NR; ++m) {
+        if constexpr (WT == W_F32) {
+#pragma unroll
+          for (int t = 0; t < NB; ++t)
+            if (t0 + t < B) out[m][t] += chunk_dot<WT>(w[m][q], ubase + (size_t)t * ub, cc * E);
+        } else if constexpr (WT == W_F16) {
+#pragma unroll
+          for (int t = 0; t < NB; ++t)
+            if (t0 + t < B) {
+              float x = 0.f, y = 0.f;
+              mdot8(w[m][q], ld_keep16(ubase + (size_t)t * ub + (size_t)cc * 16), x, y);
+              out[m][t] += x + y;
+            }
+        } else {
+          // one chunk = one 32-element group: (q - 8) pairs, then the group scale
+          const float sc = __half2float(S[m][(size_t)i * (d / 32) + cc]);
+          const uint4 p0 = q8_pairs(w[m][q].x), p1 = q8_pairs(w[m][q].y), p2 = q8_pairs(w[m][q].z),
+                      p3 = q8_pairs(w[m][q].w);
+#pragma unroll
+          for (int t = 0; t < NB; ++t)
+            if (t0 + t < B) {
+              const char *uc = ubase + (size_t)t * ub + (size_t)cc * 64;
+              float x = 0.f, y = 0.f;
+              mdot8(p0, ld_keep16(uc), x, y);
+              mdot8(p1, ld_keep16(uc + 16), x, y);
+              mdot8(p2, ld_keep16(uc + 32), x, y);
+              mdot8(p3, ld_keep16(uc + 48), x, y);
+              out[m][t] = fmaf(sc, x + y, out[m][t]);
+            }
+        }
       }
     }
   }
 #pragma unroll
-  for (int t = 0; t < NB; ++t) out[t] = warp_sum(out[t]);
+  for (int m = 0; m < NR; ++m)
+#pragma unroll
+    for (int t = 0; t < NB; ++t) out[m][t] = warp_sum(out[m][t]);
 }
 
 // 8 consecutive elements (column group g) of W2T row i, as floats
@@ -430,19 +503,21 @@ __global__ void __launch_bounds__(512) ffn_gather_kernel(FfnArgs a) {
       if (m == 0u && !dense_row) {
 #pragma unroll
         for (int t = 0; t < NB; ++t) av[t] = 0.f;
+      } else if constexpr (ACT == ACT_SWIGLU) {
+        const void *Ws[2] = {a.w_up, a.w_gate};
+        const __half *Ss[2] = {a.s_up, a.s_gate};
+        float v[2][NB];
+        row_dots<NB, WT, 2>(Ws, Ss, i, a.u, d, B, t0, lane, v);
+#pragma unroll
+        for (int t = 0; t < NB; ++t) av[t] = ((m >> t) & 1u) ? silu(v[1][t]) * v[0][t] : 0.f;
       } else {
-        float v[NB];
-        row_dot<NB, WT>(a.w_up, a.s_up, i, a.u, d, B, t0, lane, v);
-        if (ACT == ACT_SWIGLU) {
-          float g[NB];
-          row_dot<NB, WT>(a.w_gate, a.s_gate, i, a.u, d, B, t0, lane, g);
+        const void *Ws[1] = {a.w_up};
+        const __half *Ss[1] = {a.s_up};
+        float v[1][NB];
+        row_dots<NB, WT, 1>(Ws, Ss, i, a.u, d, B, t0, lane, v);
+        const float bi = a.b_up[i];
 #pragma unroll
-          for (int t = 0; t < NB; ++t) av[t] = ((m >> t) & 1u) ? silu(g[t]) * v[t] : 0.f;
-        } else {
-          const float bi = a.b_up[i];
-#pragma unroll
-          for (int t = 0; t < NB; ++t) av[t] = ((m >> t) & 1u) ? fmaxf(v[t] + bi, 0.f) : 0.f;
-        }
+        for (int t = 0; t < NB; ++t) av[t] = ((m >> t) & 1u) ? fmaxf(v[0][t] + bi, 0.f) : 0.f;
       }
       if (lane == 0) {
 #pragma unroll

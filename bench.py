@@ -67,6 +67,8 @@ def parse(argv=None):
     ap.add_argument("--ref-seconds", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--json-out", default=None)
+    ap.add_argument("--stack", action="store_true",
+                    help="time pi_decode_ffn_stack through all layers of a stacked config (tokens/s)")
     return ap.parse_args(argv)
 
 
@@ -430,11 +432,105 @@ def bench_ours(args, world, rank, local):
     return line
 
 
+def bench_stack(args, world, rank, local):
+    """FFN-stack decode: every layer of a stacked config (RMS norm, predictor,
+    sparse FFN, residual add), one token batch per pass, timed with CUDA
+    events around graph replays.  Attention is not part of the path."""
+    from activation_sparse_decode_gemv_b200 import binding as pb
+    assert torch.cuda.is_available(), "bench.py needs a CUDA device"
+    pb.lib()
+    dev = torch.device("cuda", local)
+    cfg = inputs.CONFIGS[args.config]
+    assert cfg.stacked, f"{cfg.name} is not a stacked config"
+    B, L, T = args.batch, cfg.n_layers, args.tokens
+    seed = 3000 + rank
+    t0 = time.perf_counter()
+    layers = [inputs.make_layer(cfg, l, seed=seed, device=dev) for l in range(L)]
+    gen_s = time.perf_counter() - t0
+    handles = [pb.FfnLayer.from_tensors(lt) for lt in layers]
+    ws = pb.make_workspace(handles, B, dev)
+    xs = [inputs.make_tokens(cfg, t, B, seed=seed).to(dev) for t in range(T)]
+    x = torch.empty_like(xs[0])
+    stream = torch.cuda.Stream(dev)
+    # bytes per pass from the stack's own traces (untimed)
+    idx = torch.empty((L, B, cfg.f), dtype=torch.int32, device=dev)
+    cnt = torch.empty((L, B), dtype=torch.int32, device=dev)
+    tok_bytes = []
+    for t in range(T):
+        x.copy_(xs[t])
+        pb.pi_decode_ffn_stack(handles, x, ws, idx_trace=idx, count_trace=cnt, flags=args.flags)
+        torch.cuda.synchronize()
+        c = cnt.cpu()
+        nb = 0
+        for l in range(L):
+            sets = [idx[l, b, :int(c[l, b])].long() for b in range(B)]
+            union = torch.unique(torch.cat(sets)) if int(c[l].sum()) else torch.empty(0, dtype=torch.long)
+            nb += step_bytes(cfg, B, len(union))
+        tok_bytes.append(nb)
+    assert pb.pi_get_device_status(ws) == 0
+    graphs = []
+    for t in range(T):
+        with torch.cuda.stream(stream):
+            x.copy_(xs[t])
+            pb.pi_decode_ffn_stack(handles, x, ws, flags=args.flags, stream=stream)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            x.copy_(xs[t])
+            pb.pi_decode_ffn_stack(handles, x, ws, flags=args.flags, stream=stream)
+        graphs.append(g)
+
+    def run(n):
+        with torch.cuda.stream(stream):
+            for j in range(n):
+                graphs[j % T].replay()
+
+    run(args.warmup)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        run(args.steps)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    sec = ev0.elapsed_time(ev1) / 1e3
+    assert pb.pi_get_device_status(ws) == 0
+    nbytes = sum(tok_bytes[j % T] for j in range(args.steps))
+    gbs, tmax = aggregate(nbytes, sec, world)
+    peaks = {}
+    pp = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(pp):
+        peaks = json.load(open(pp))
+    peak = peaks.get("hbm_gbs", 6650.0)
+    return {
+        "metric": "FFN-stack decode tokens/s (attention excluded)",
+        "value": B * args.steps / tmax * world, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": tmax / args.steps * 1e3, "us_per_layer": tmax / args.steps / L * 1e6,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "weights": cfg.wtype,
+        "data": "synthetic",
+        "config": {"workload": f"{cfg.name}: {L}-layer FFN stack d={cfg.d} f={cfg.f} r={cfg.r} {cfg.act} "
+                               f"{cfg.wtype} weights, batch {B}",
+                   "batch": B, "layers": L, "tokens": T, "weights_gb": sum(l.nbytes() for l in layers) / 1e9,
+                   "bytes_per_step": nbytes / args.steps, "generation_s": gen_s},
+        "roofline": {"bound": "hbm", "achieved": gbs / world, "peak": peak, "unit": "GB/s",
+                     "frac": gbs / world / peak, "peak_source": "measured" if "hbm_gbs" in peaks else "fallback"},
+        "clocks": clk.summary(),
+    }
+
+
 def main(argv=None):
     args = parse(argv)
     world, rank, local = dist_init()
     try:
-        line = bench_reference(args, world, rank) if args.impl == "reference" else bench_ours(args, world, rank, local)
+        if args.impl == "reference":
+            line = bench_reference(args, world, rank)
+        elif args.stack:
+            line = bench_stack(args, world, rank, local)
+        else:
+            line = bench_ours(args, world, rank, local)
         if rank == 0 and line is not None:
             s = json.dumps(line)
             print(s, flush=True)
