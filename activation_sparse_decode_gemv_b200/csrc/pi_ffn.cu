@@ -581,10 +581,26 @@ cudaError_t fused_launch(const F::Args &a, int G, cudaStream_t st) {
   cfg.blockDim = dim3(F::kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute at[1];
+  // cooperative (all CTAs co-resident for the grid barriers) and, where the
+  // runtime accepts the pair, programmatic dependent launch
+  static int pdl_ok = -1;
+  cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeCooperative;
   at[0].val.cooperative = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
+  if (pdl_ok != 0) {
+    cfg.numAttrs = 2;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, F::decode_fused_kernel<WT, ACT, CPT>, a);
+    if (e == cudaSuccess) {
+      pdl_ok = 1;
+      return e;
+    }
+    if (pdl_ok == 1) return e;
+    cudaGetLastError();
+    pdl_ok = 0;
+  }
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, F::decode_fused_kernel<WT, ACT, CPT>, a);
 }

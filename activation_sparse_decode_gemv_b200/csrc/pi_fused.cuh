@@ -533,10 +533,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Args a) {
   for (int k = tid; k < kMaxOwnTiles; k += blockDim.x) S.own_bits[k] = 0u;
   __syncthreads();
 
+  // Programmatic dependent launch: the next step's grid may be scheduled
+  // now, and its CTAs take SMs as this grid's CTAs leave.  The producer
+  // streams weights only (P1 rows, P2 tiles, weight rows), which no earlier
+  // kernel writes, so it starts at once; the consumers wait for the
+  // preceding grid before reading the input or touching the workspace.
+  pdl_launch_dependents();
   if (warp == kConsumerWarps) {
     producer<WT, ACT>(S, a, c, G, lane);
     return;
   }
+  pdl_wait();
 
   // ------------------------------------------------------------ consumers
   const int nch = d / EC;
