@@ -504,8 +504,11 @@ pi_status run_predict_tc(const pi_ffn *h, const void *u, int B, int32_t *idx, in
   b.ctr = w.ctr_p2();
   b.status = w.status();
   PI_CUDA((ts_launch<TC::K_P2, pi::W_F16, 0>(b, G, st)));
-  PI_CUDA(launch(pi::compact_kernel, dim3(B + 1), dim3(1024), st, (const uint32_t *)w.mask(), h->nwords, idx_stride, B,
-                 idx, count, w.uwords(), w.uprefix(), w.ulist(), w.ucount()));
+  // the tensor-core FFN kernels list their tiles from the mask words; the
+  // compaction runs only for the caller's id lists
+  if (idx || count)
+    PI_CUDA(launch(pi::compact_kernel, dim3(B + 1), dim3(1024), st, (const uint32_t *)w.mask(), h->nwords, idx_stride,
+                   B, idx, count, w.uwords(), w.uprefix(), w.ulist(), w.ucount()));
   return PI_OK;
 }
 
@@ -520,7 +523,6 @@ pi_status run_ffn_tc(const pi_ffn *h, const void *u, int B, float *out, int accu
   a.tm1 = h->tm_gate;
   a.ts0 = h->ts_up;
   a.ts1 = h->ts_gate;
-  a.uwords = w.uwords();
   a.nrows = D.d_ffn;
   a.K = D.d_model;
   a.img0 = D.wtype == PI_W_INT4G32 ? w.uimg_perm() : w.uimg();
@@ -544,7 +546,7 @@ pi_status run_ffn_tc(const pi_ffn *h, const void *u, int B, float *out, int accu
   TC::DownArgs dn{};
   dn.tm = h->tm_down;
   dn.ts = h->ts_down;
-  dn.uwords = w.uwords();
+  dn.mask = w.mask();
   dn.nwords = h->nwords;
   dn.f = D.d_ffn;
   dn.d = D.d_model;

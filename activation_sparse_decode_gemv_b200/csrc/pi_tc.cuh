@@ -345,18 +345,30 @@ PI_DEV void ctrl_init(TcCtrl &C, unsigned nw, unsigned empty_count) {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
-// All threads: list the 128-neuron tiles that hold a set bit of the union
-// words (4 words per tile), in ascending order, into C.tlist / C.n_tiles.
-PI_DEV void list_tiles(TcCtrl &C, const uint32_t *uwords, int nwords, int n_all) {
+// All threads: list the 128-neuron tiles that hold a set bit of any token's
+// mask words (4 words per tile, B tokens), in ascending order, into C.tlist /
+// C.n_tiles.
+PI_DEV void list_tiles(TcCtrl &C, const uint32_t *mask, int nwords, int B, int n_all) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nthreads = blockDim.x;
   int base = 0;
   for (int t0 = 0; t0 < n_all; t0 += nthreads) {
     const int t = t0 + tid;
     bool act = false;
     if (t < n_all) {
+      uint32_t any = 0u;
+      for (int b0 = 0; b0 < B; b0 += 4) {
+        uint32_t v[4][4];
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        if (4 * t + k < nwords) act |= __ldg(uwords + 4 * t + k) != 0u;
+        for (int bb = 0; bb < 4; ++bb)
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            v[bb][k] = (b0 + bb < B && 4 * t + k < nwords) ? __ldcg(mask + (size_t)(b0 + bb) * nwords + 4 * t + k) : 0u;
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb)
+#pragma unroll
+          for (int k = 0; k < 4; ++k) any |= v[bb][k];
+      }
+      act = any != 0u;
     }
     const unsigned bal = __ballot_sync(0xffffffffu, act);
     if (lane == 0) C.wcnt[warp] = __popc(bal);
@@ -452,7 +464,6 @@ struct RowArgs {
   CUtensorMap tm0, tm1;         // row data of matrix 0 / 1: fp16 [rows x K] (box 64 x 128) or
                                 // packed int4 bytes [rows x K/2] (box 128 x 128)
   CUtensorMap ts0, ts1;         // int4 scale bytes [rows x K/16] (box 16 x 128)
-  const uint32_t *uwords;       // ffn_up: union mask words (a tile runs when one of its 4 words is set)
   int nrows;                    // rows of the matrices
   int K;                        // row length (elements)
   const unsigned char *img0;    // B operand image (u, or h_hi)
@@ -519,7 +530,7 @@ __global__ void __launch_bounds__(RowShape<KIND, WT, ACT>::THREADS, 1) row_gemm_
 
   const int T_all = (a.nrows + kM - 1) / kM;
   if (KIND == K_UP) {
-    list_tiles(C, a.uwords, a.nwords, T_all);
+    list_tiles(C, a.mask, a.nwords, a.B, T_all);
   } else if (tid == 0) {
     C.n_tiles = T_all;
   }
@@ -770,7 +781,7 @@ __global__ void __launch_bounds__(RowShape<KIND, WT, ACT>::THREADS, 1) row_gemm_
 struct DownArgs {
   CUtensorMap tm;               // W2T: fp16 [f x d] (box 64 x 64) or packed int4 bytes [f x d/2] (box 128 x 64)
   CUtensorMap ts;               // int4 scale bytes [f x d/16] (box 16 x 64)
-  const uint32_t *uwords;       // union mask words (the same tile list as ffn_up)
+  const uint32_t *mask;         // per-token mask words [B x nwords] (the same tile list as ffn_up)
   int nwords, f, d, B;
   const unsigned char *aimg;    // a image, K = the listed tiles' neurons
   float *y;                     // [B x d]
@@ -822,7 +833,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_down_kernel(const __grid_cons
   pdl_wait();
   pdl_launch_dependents();
 
-  list_tiles(C, a.uwords, a.nwords, (a.f + kM - 1) / kM);
+  list_tiles(C, a.mask, a.nwords, a.B, (a.f + kM - 1) / kM);
   const int d = a.d;
   const long long T = (d + kDownTileD - 1) / kDownTileD;
   const long long SK = (long long)C.n_tiles * (kM / kDownStepK);
