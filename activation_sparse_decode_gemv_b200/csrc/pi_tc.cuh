@@ -57,6 +57,7 @@ constexpr int kDownStepK = 64;         // neurons per down-projection step
 constexpr int kMaxTiles = 1024;        // 128-neuron tiles the ffn kernels can list (d_ffn <= 131072)
 constexpr int kImgStep = 128;          // token images are padded to a multiple of 128 in K
 constexpr uint32_t kSw128 = 2;         // UMMA descriptor layout code of the 128-byte swizzle
+constexpr int kMaxSlots = 12;          // deepest ring (bytes in flight per SM are what hide the latency)
 constexpr unsigned long long kWaitNs = 2000000000ull;
 
 enum Kind { K_P1 = 0, K_P2 = 1, K_UP = 2 };
@@ -312,7 +313,7 @@ __global__ void __launch_bounds__(256) u_image_kernel(const __half *__restrict__
 
 // ---------------------------------------------------------------- shared pieces
 struct TcCtrl {
-  uint64_t full[6], empty[6];
+  uint64_t full[kMaxSlots], empty[kMaxSlots];
   uint64_t afull[2], afree[2], accfull[2], accfree[2];
   uint64_t wbar;  // the 256 worker threads' barrier (stream-K fix-up)
   uint32_t tmem;
@@ -491,7 +492,7 @@ struct RowShape {
   static constexpr int IMG_OFF = NMAT * (ABOX + SBOX);
   static constexpr int SLOTB = (IMG_OFF + IMGB + 1023) / 1024 * 1024;
   static constexpr int NSLOT_FIT = kSmemBudget / SLOTB;
-  static constexpr int NSLOT = NSLOT_FIT > 6 ? 6 : NSLOT_FIT;
+  static constexpr int NSLOT = NSLOT_FIT > kMaxSlots ? kMaxSlots : NSLOT_FIT;
   static constexpr int TX = IMG_OFF + IMGB;         // bytes landing per unit
   static constexpr int CTRL_OFF = NSLOT * SLOTB;
   static constexpr int SMEM = CTRL_OFF + kCtrlBytes + 1024;  // + alignment slack
@@ -803,7 +804,7 @@ struct DownShape {
   static constexpr int SLOTB = (IMG_OFF + IMGB + 1023) / 1024 * 1024;
   static constexpr int ABUF = Q4 ? kDownStepK * kDownTileD * 2 : 0;  // int4: dequantised canonical A, 32 KB
   static constexpr int NSLOT_FIT = (kSmemBudget - 2 * ABUF) / SLOTB;
-  static constexpr int NSLOT = NSLOT_FIT > 6 ? 6 : NSLOT_FIT;
+  static constexpr int NSLOT = NSLOT_FIT > kMaxSlots ? kMaxSlots : NSLOT_FIT;
   static constexpr int TX = IMG_OFF + IMGB;
   static constexpr int A_OFF = NSLOT * SLOTB;
   static constexpr int CTRL_OFF = A_OFF + 2 * ABUF;

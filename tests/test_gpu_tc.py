@@ -101,6 +101,22 @@ def test_tc_determinism_bitwise(cuda_device):
         assert torch.equal(t1, t2)
 
 
+def test_tc_decode_without_id_lists(cuda_device):
+    """pi_decode_ffn at B >= 16 without idx/count (the compaction is then
+    skipped; the FFN kernels list their tiles from the mask words) gives the
+    same y, bitwise, as the call that also returns the id lists."""
+    cfg = inputs.CONFIGS["llama70b_swiglu_int4"].scaled(**SMALL)
+    lt = inputs.make_layer(cfg, 0, seed=9)
+    g = Gpu(lt, 32)
+    u = inputs.layer_input(cfg, inputs.make_tokens(cfg, 0, 24, seed=9)).cuda()
+    y1, _, _ = g.decode(u)
+    y2 = torch.full_like(y1, float("nan"))
+    pb.pi_decode_ffn(g.layer, u, y2, g.ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    assert g.status() == 0
+
+
 def test_tc_stack_composes_layers(cuda_device):
     """pi_decode_ffn_stack over 3 layers at B=16 equals three one-layer stack
     calls bitwise, traces included (the layer loop adds nothing of its own;
