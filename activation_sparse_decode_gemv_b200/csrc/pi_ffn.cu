@@ -485,6 +485,8 @@ pi_status run_predict_tc(const pi_ffn *h, const void *u, int B, int32_t *idx, in
   a.img0 = w.uimg();
   a.out0 = w.himg_hi();
   a.out1 = w.himg_lo();
+  a.uwords = w.uwords();
+  a.nwords = h->nwords;
   a.B = B;
   a.part = w.tc_part();
   a.ctr = w.ctr_p1();
@@ -498,14 +500,15 @@ pi_status run_predict_tc(const pi_ffn *h, const void *u, int B, int32_t *idx, in
   b.img1 = w.himg_lo();
   b.bias = D.p_bias;
   b.mask_out = w.mask();
+  b.uwords = w.uwords();
   b.nwords = h->nwords;
   b.B = B;
   b.part = w.tc_part();
   b.ctr = w.ctr_p2();
   b.status = w.status();
   PI_CUDA((ts_launch<TC::K_P2, pi::W_F16, 0>(b, G, st)));
-  // the tensor-core FFN kernels list their tiles from the mask words; the
-  // compaction runs only for the caller's id lists
+  // pred_h clears and pred_s sets the union words the tensor-core FFN kernels
+  // list their tiles from; the compaction runs only for the caller's id lists
   if (idx || count)
     PI_CUDA(launch(pi::compact_kernel, dim3(B + 1), dim3(1024), st, (const uint32_t *)w.mask(), h->nwords, idx_stride,
                    B, idx, count, w.uwords(), w.uprefix(), w.ulist(), w.ucount()));
@@ -523,6 +526,7 @@ pi_status run_ffn_tc(const pi_ffn *h, const void *u, int B, float *out, int accu
   a.tm1 = h->tm_gate;
   a.ts0 = h->ts_up;
   a.ts1 = h->ts_gate;
+  a.uwords = w.uwords();
   a.nrows = D.d_ffn;
   a.K = D.d_model;
   a.img0 = D.wtype == PI_W_INT4G32 ? w.uimg_perm() : w.uimg();
@@ -546,7 +550,7 @@ pi_status run_ffn_tc(const pi_ffn *h, const void *u, int B, float *out, int accu
   TC::DownArgs dn{};
   dn.tm = h->tm_down;
   dn.ts = h->ts_down;
-  dn.mask = w.mask();
+  dn.uwords = w.uwords();
   dn.nwords = h->nwords;
   dn.f = D.d_ffn;
   dn.d = D.d_model;

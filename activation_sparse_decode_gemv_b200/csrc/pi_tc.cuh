@@ -346,30 +346,19 @@ PI_DEV void ctrl_init(TcCtrl &C, unsigned nw, unsigned empty_count) {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
-// All threads: list the 128-neuron tiles that hold a set bit of any token's
-// mask words (4 words per tile, B tokens), in ascending order, into C.tlist /
-// C.n_tiles.
-PI_DEV void list_tiles(TcCtrl &C, const uint32_t *mask, int nwords, int B, int n_all) {
+// All threads: list the 128-neuron tiles that hold a set bit of the union
+// words (4 words per tile: the OR of the tokens' mask words), in ascending
+// order, into C.tlist / C.n_tiles.
+PI_DEV void list_tiles(TcCtrl &C, const uint32_t *uwords, int nwords, int n_all) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nthreads = blockDim.x;
   int base = 0;
   for (int t0 = 0; t0 < n_all; t0 += nthreads) {
     const int t = t0 + tid;
     bool act = false;
     if (t < n_all) {
-      uint32_t any = 0u;
-      for (int b0 = 0; b0 < B; b0 += 4) {
-        uint32_t v[4][4];
 #pragma unroll
-        for (int bb = 0; bb < 4; ++bb)
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            v[bb][k] = (b0 + bb < B && 4 * t + k < nwords) ? __ldcg(mask + (size_t)(b0 + bb) * nwords + 4 * t + k) : 0u;
-#pragma unroll
-        for (int bb = 0; bb < 4; ++bb)
-#pragma unroll
-          for (int k = 0; k < 4; ++k) any |= v[bb][k];
-      }
-      act = any != 0u;
+      for (int k = 0; k < 4; ++k)
+        if (4 * t + k < nwords) act |= __ldcg(uwords + 4 * t + k) != 0u;
     }
     const unsigned bal = __ballot_sync(0xffffffffu, act);
     if (lane == 0) C.wcnt[warp] = __popc(bal);
@@ -472,6 +461,7 @@ struct RowArgs {
   const float *bias;            // pred_s: predictor bias; ffn_up ReLU: b_up
   const uint32_t *mask;         // ffn_up: per-token mask words [B x nwords]
   uint32_t *mask_out;           // pred_s: per-token mask words [B x nwords]
+  uint32_t *uwords;             // pred_h: zeroed; pred_s: OR of the tokens' mask words; ffn_up: read
   int nwords, B;
   unsigned char *out0, *out1;   // pred_h: h_hi / h_lo images; ffn_up: a image
   float *part;                  // stream-K partials [G x 2 x kPartFloats]
@@ -499,7 +489,7 @@ struct RowShape {
   static constexpr int ACC_COLS = NMAT * kN;        // per accumulator buffer
   static constexpr int A_COLS = NMAT * 64;          // int4: per tensor-memory A buffer (128 K)
   static constexpr uint32_t TMEM_COLS = Q4 ? 512 : 128;
-  static constexpr int NW = Q4 ? 16 : 8;            // worker warps
+  static constexpr int NW = 8;                      // worker warps
   static constexpr int THREADS = 64 + 32 * NW;
   static constexpr int KQ = NW / 4;                 // workers per tensor-memory lane quarter
   static constexpr int TOKW = kN / KQ;              // epilogue token columns per worker
@@ -531,10 +521,12 @@ __global__ void __launch_bounds__(RowShape<KIND, WT, ACT>::THREADS, 1) row_gemm_
 
   const int T_all = (a.nrows + kM - 1) / kM;
   if (KIND == K_UP) {
-    list_tiles(C, a.mask, a.nwords, a.B, T_all);
+    list_tiles(C, a.uwords, a.nwords, T_all);
   } else if (tid == 0) {
     C.n_tiles = T_all;
   }
+  if (KIND == K_P1 && a.uwords)  // cleared here, set by pred_s (the next kernel)
+    for (int w = cta * S::THREADS + tid; w < a.nwords; w += G * S::THREADS) a.uwords[w] = 0u;
   __syncthreads();
   const long long T = C.n_tiles;
   const long long SK = (a.K + S::STEPK - 1) / S::STEPK;
@@ -663,25 +655,31 @@ __global__ void __launch_bounds__(RowShape<KIND, WT, ACT>::THREADS, 1) row_gemm_
             fine = false;
             break;
           }
-          // this thread: row m, the 32-element group g of the unit (one 16-byte chunk)
-          const int g = sub * 4 + kq;
-          const uint32_t acol = lane_base + (uint32_t)(2 * S::ACC_COLS + b * S::A_COLS + kq * 16);
+          // this thread: row m, GPS consecutive 32-element groups of the unit
+          // (one 16-byte chunk each), GPS = 4 / KQ
+          constexpr int GPS = 4 / S::KQ;
 #pragma unroll
-          for (int mat = 0; mat < S::NMAT; ++mat) {
-            // packed row m of the swizzled box: 16-byte chunk g sits at (g ^ (m % 8)) * 16
-            const uint4 pk = *reinterpret_cast<const uint4 *>(slot + mat * S::ABOX + m * 128 + ((g ^ (m & 7)) << 4));
-            const __half sc = *reinterpret_cast<const __half *>(slot + S::SC_OFF + mat * S::SBOX + m * 16 + g * 2);
-            const __half2 s2 = __halves2half2(sc, sc);
-            const uint32_t wds[4] = {pk.x, pk.y, pk.z, pk.w};
-            uint32_t v[16];
+          for (int gg = 0; gg < GPS; ++gg) {
+            const int g = sub * 4 + kq * GPS + gg;
+            const uint32_t acol = lane_base + (uint32_t)(2 * S::ACC_COLS + b * S::A_COLS + (kq * GPS + gg) * 16);
 #pragma unroll
-            for (int t = 0; t < 4; ++t) {
-              uint32_t o[4];
-              q8_to_h4_paired(wds[t], s2, o);
+            for (int mat = 0; mat < S::NMAT; ++mat) {
+              // packed row m of the swizzled box: 16-byte chunk g sits at (g ^ (m % 8)) * 16
+              const uint4 pk =
+                  *reinterpret_cast<const uint4 *>(slot + mat * S::ABOX + m * 128 + ((g ^ (m & 7)) << 4));
+              const __half sc = *reinterpret_cast<const __half *>(slot + S::SC_OFF + mat * S::SBOX + m * 16 + g * 2);
+              const __half2 s2 = __halves2half2(sc, sc);
+              const uint32_t wds[4] = {pk.x, pk.y, pk.z, pk.w};
+              uint32_t v[16];
 #pragma unroll
-              for (int c = 0; c < 4; ++c) v[t * 4 + c] = o[c];
+              for (int t = 0; t < 4; ++t) {
+                uint32_t o[4];
+                q8_to_h4_paired(wds[t], s2, o);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) v[t * 4 + c] = o[c];
+              }
+              tmem_st16(acol + mat * 64, v);
             }
-            tmem_st16(acol + mat * 64, v);
           }
           tmem_wait_st();
           tc_fence_before();
@@ -743,12 +741,17 @@ __global__ void __launch_bounds__(RowShape<KIND, WT, ACT>::THREADS, 1) row_gemm_
         const bool valid = row < a.nrows;
         const float bias = valid ? __ldg(a.bias + row) : 0.f;
         const int word = (int)(j_tile * kM + q * 32) >> 5;
+        unsigned any = 0u;
 #pragma unroll
         for (int j = 0; j < S::TOKW; ++j) {
           const int n = kq * S::TOKW + j;
           const unsigned bits = __ballot_sync(0xffffffffu, valid && (v[j] + bias > 0.f));
-          if (lane == 0 && n < a.B && word < a.nwords) a.mask_out[(size_t)n * a.nwords + word] = bits;
+          if (lane == 0 && n < a.B && word < a.nwords) {
+            a.mask_out[(size_t)n * a.nwords + word] = bits;
+            any |= bits;
+          }
         }
+        if (lane == 0 && any) atomicOr(a.uwords + word, any);  // union words (order-free)
       } else {
         // a image position: listed tile j_tile, row m
         const bool valid = row < a.nrows;
@@ -782,7 +785,7 @@ __global__ void __launch_bounds__(RowShape<KIND, WT, ACT>::THREADS, 1) row_gemm_
 struct DownArgs {
   CUtensorMap tm;               // W2T: fp16 [f x d] (box 64 x 64) or packed int4 bytes [f x d/2] (box 128 x 64)
   CUtensorMap ts;               // int4 scale bytes [f x d/16] (box 16 x 64)
-  const uint32_t *mask;         // per-token mask words [B x nwords] (the same tile list as ffn_up)
+  const uint32_t *uwords;       // union mask words (the same tile list as ffn_up)
   int nwords, f, d, B;
   const unsigned char *aimg;    // a image, K = the listed tiles' neurons
   float *y;                     // [B x d]
@@ -834,7 +837,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_down_kernel(const __grid_cons
   pdl_wait();
   pdl_launch_dependents();
 
-  list_tiles(C, a.mask, a.nwords, a.B, (a.f + kM - 1) / kM);
+  list_tiles(C, a.uwords, a.nwords, (a.f + kM - 1) / kM);
   const int d = a.d;
   const long long T = (d + kDownTileD - 1) / kDownTileD;
   const long long SK = (long long)C.n_tiles * (kM / kDownStepK);
