@@ -135,7 +135,15 @@ pi_status pi_sparse_ffn(pi_ffn_t h, const void *u, int B, const int32_t *idx, co
                         unsigned flags, void *ws, size_t ws_bytes, pi_stream_t stream);
 
 /* Whole single-layer decode step (steps 1-4) from the FFN input u.  y: [B x d]
- * fp32.  idx/count: optional outputs as in pi_predict (NULL to skip). */
+ * fp32.  idx/count: optional outputs as in pi_predict (NULL to skip).
+ * Execution (the same for the predictor and sparse-FFN entry points where it
+ * applies):
+ *  - batch 1, fp16/int4 weights (d <= 8192): one persistent fused kernel;
+ *  - batch 16..32, fp16 predictor, fp16 or int4 weights (int4: d % 256 == 0):
+ *    tensor-core GEMMs over the 128-neuron tiles that hold a predicted neuron
+ *    of some token;
+ *  - otherwise: CUDA-core predictor, compaction, gather and reduction kernels.
+ * Results agree within the stated tolerances whichever path runs. */
 pi_status pi_decode_ffn(pi_ffn_t h, const void *u, int B, float *y, int32_t *idx, int32_t *count, unsigned flags,
                         void *ws, size_t ws_bytes, pi_stream_t stream);
 
