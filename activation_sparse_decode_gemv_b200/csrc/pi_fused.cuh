@@ -261,6 +261,19 @@ PI_DEV void dot16_q_mixed(const uint2 &w, const uint4 &u0, const uint4 &u1, floa
   dot8_mixed(make_uint4(q[4], q[5], q[6], q[7]), u1, x, y);
 }
 
+// the 8 int4 codes n0..n7 of one 32-bit word as the fp16 pairs (1024 + n_j,
+// 1024 + n_(j+4)), j = 0..3: one shift and one masked OR per pair (0x6400 | q
+// is the fp16 value 1024 + q)
+PI_DEV uint4 q8_pairs_biased(uint32_t w) {
+  return make_uint4((w & 0x000F000Fu) | 0x64006400u, ((w >> 4) & 0x000F000Fu) | 0x64006400u,
+                    ((w >> 8) & 0x000F000Fu) | 0x64006400u, ((w >> 12) & 0x000F000Fu) | 0x64006400u);
+}
+// fp16 pairs (k, k+4) of each 8-element block of 8 fp16 inputs (16 B)
+PI_DEV uint4 pair_k4(const uint4 &v) {
+  return make_uint4(__byte_perm(v.x, v.z, 0x5410), __byte_perm(v.x, v.z, 0x7632), __byte_perm(v.y, v.w, 0x5410),
+                    __byte_perm(v.y, v.w, 0x7632));
+}
+
 // sum N independent values across the warp; the N butterflies are
 // interleaved so that their shuffles overlap
 template <int N>
@@ -601,6 +614,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Args a) {
       }
     }
   }
+  // int4 dots take u in the (k, k+4) pair order of q8_pairs_biased, and the
+  // chunk sums of u for the 1032 (= 1024 + 8) bias of the unpacked codes
+  uint4 up4[CPT][UW];
+  float usum[CPT];
+#pragma unroll
+  for (int q = 0; q < CPT; ++q) {
+    usum[q] = 0.f;
+#pragma unroll
+    for (int j = 0; j < UW; ++j) {
+      up4[q][j] = WT == W_INT4 ? pair_k4(uh[q][j]) : uh[q][j];
+      if (WT == W_INT4) {
+        const __half2 *hp = reinterpret_cast<const __half2 *>(&uh[q][j]);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f = __half22float2(hp[k]);
+          usum[q] += f.x;
+          usum[q] += f.y;
+        }
+      }
+    }
+  }
   float y[CPT][EC];
 #pragma unroll
   for (int q = 0; q < CPT; ++q)
@@ -753,16 +787,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Args a) {
           if (ACT == ACT_SWIGLU)
             dot8_mixed(*reinterpret_cast<const uint4 *>(nd[g] + NL.gate + coff[cq] * 16), uh[cq][0], gx, gy);
         } else {
+          // sum_k (q_k - 8) u_k = sum_k (1024 + q_k) u_k - 1032 sum_k u_k; the
+          // products of two fp16 values are exact in fp32
           const float su = __half2float(*reinterpret_cast<const __half *>(nd[g] + NL.sup + (coff[cq] >> 1) * 2));
+          const uint2 wu = *reinterpret_cast<const uint2 *>(nd[g] + NL.up + coff[cq] * 8);
           float x = 0.f, yv = 0.f;
-          dot16_q_mixed(*reinterpret_cast<const uint2 *>(nd[g] + NL.up + coff[cq] * 8), uh[cq][0], uh[cq][1], x, yv);
-          ux = fmaf(su, x + yv, ux);
+          dot8_mixed(q8_pairs_biased(wu.x), up4[cq][0], x, yv);
+          dot8_mixed(q8_pairs_biased(wu.y), up4[cq][1], x, yv);
+          ux = fmaf(su, fmaf(-1032.f, usum[cq], x + yv), ux);
           if (ACT == ACT_SWIGLU) {
             const float sg = __half2float(*reinterpret_cast<const __half *>(nd[g] + NL.sgate + (coff[cq] >> 1) * 2));
+            const uint2 wg = *reinterpret_cast<const uint2 *>(nd[g] + NL.gate + coff[cq] * 8);
             float x2 = 0.f, y2 = 0.f;
-            dot16_q_mixed(*reinterpret_cast<const uint2 *>(nd[g] + NL.gate + coff[cq] * 8), uh[cq][0], uh[cq][1], x2,
-                          y2);
-            gx = fmaf(sg, x2 + y2, gx);
+            dot8_mixed(q8_pairs_biased(wg.x), up4[cq][0], x2, y2);
+            dot8_mixed(q8_pairs_biased(wg.y), up4[cq][1], x2, y2);
+            gx = fmaf(sg, fmaf(-1032.f, usum[cq], x2 + y2), gx);
           }
         }
       }
@@ -835,14 +874,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Args a) {
           const float sd = __half2float(*reinterpret_cast<const __half *>(ndg + NL.sdown + (coff[cq] >> 1) * 2));
           const uint2 wq = *reinterpret_cast<const uint2 *>(ndg + NL.down + coff[cq] * 8);
           const float as = ag * sd;
-          uint32_t qh[8];
-          q8_to_h2(wq.x, qh);
-          q8_to_h2(wq.y, qh + 4);
+          // (q - 8) exactly, as the pairs (j, j + 4) of each 8-element word
+          const __half2 off = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));
+          const uint4 p0 = q8_pairs_biased(wq.x), p1 = q8_pairs_biased(wq.y);
+          const uint32_t pw[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
 #pragma unroll
           for (int kq = 0; kq < 8; ++kq) {
-            const float2 v = __half22float2(*reinterpret_cast<const __half2 *>(&qh[kq]));
-            y[cq][2 * kq] = fmaf(as, v.x, y[cq][2 * kq]);
-            y[cq][2 * kq + 1] = fmaf(as, v.y, y[cq][2 * kq + 1]);
+            const __half2 hv = __hsub2(*reinterpret_cast<const __half2 *>(&pw[kq]), off);
+            const float2 v = __half22float2(hv);
+            const int e = (kq >> 2) * 8 + (kq & 3);  // elements e and e + 4 of the chunk
+            y[cq][e] = fmaf(as, v.x, y[cq][e]);
+            y[cq][e + 4] = fmaf(as, v.y, y[cq][e + 4]);
           }
         }
       }
