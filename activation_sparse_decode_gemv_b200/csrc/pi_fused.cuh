@@ -735,34 +735,32 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Args a) {
       break;
     }
     if (type == IT_P2) {
-      // rows warp + 8 q of the tile, two rows at a time
+      // rows warp + 8 q of the tile: all of this warp's loads first, then the
+      // dots, then one butterfly over the row sums
       const int kl = S.meta[s].first, rows = S.meta[s].n;
       constexpr int RPW = kTN / kConsumerWarps;
       unsigned b = 0u;
-#pragma unroll 1
-      for (int rp = 0; rp < RPW; rp += 2) {
-        uint4 wv[2][4];
+      uint4 wv[RPW][4];
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          const int row_i = warp + (rp + q) * kConsumerWarps;
-          const __half *row = reinterpret_cast<const __half *>(S.ring[s]) + (size_t)min(row_i, rows - 1) * r;
+      for (int q = 0; q < RPW; ++q) {
+        const int row_i = warp + q * kConsumerWarps;
+        const __half *row = reinterpret_cast<const __half *>(S.ring[s]) + (size_t)min(row_i, rows - 1) * r;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) wv[q][kk] = *reinterpret_cast<const uint4 *>(row + hoff[kk] * 8);
-        }
-        float sv[2];
+        for (int kk = 0; kk < 4; ++kk) wv[q][kk] = *reinterpret_cast<const uint4 *>(row + hoff[kk] * 8);
+      }
+      float sv[RPW];
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          float acc[4];
+      for (int q = 0; q < RPW; ++q) {
+        float acc[4];
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) acc[kk] = dot8_h2(wv[q][kk], hreg[kk]);
-          sv[q] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-        }
-        warp_sum_n<2>(sv);
+        for (int kk = 0; kk < 4; ++kk) acc[kk] = dot8_h2(wv[q][kk], hreg[kk]);
+        sv[q] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+      }
+      warp_sum_n<RPW>(sv);
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          const int row_i = warp + (rp + q) * kConsumerWarps;
-          if (row_i < rows && sv[q] + S.own_pbias[kl][row_i] > 0.f) b |= 1u << row_i;
-        }
+      for (int q = 0; q < RPW; ++q) {
+        const int row_i = warp + q * kConsumerWarps;
+        if (row_i < rows && sv[q] + S.own_pbias[kl][row_i] > 0.f) b |= 1u << row_i;
       }
       if (lane == 0 && b) {
         atomicOr(&S.tbits[s], b);
@@ -856,23 +854,48 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Args a) {
         }
       }
     }
-    // down-projection rows: y += a_g * W2T_g (every thread, its own chunks);
-    // a_g is the same in every thread, so skipping zeros never diverges
-#pragma unroll 1
-    for (int g = 0; g < ng; ++g) {
-      const float ag = __shfl_sync(0xffffffffu, a_l, 8 * g);
-      if (ag == 0.f) continue;
-      const uint8_t *ndg = S.ring[s] + g * NL.bytes;
+    // down-projection rows: y += a_g * W2T_g (every thread, its own chunks).
+    // The rows of all the item's neurons are loaded first (neurons past the
+    // item alias neuron 0); a_g is the same in every thread, so skipping the
+    // zeros never diverges.
+    float agv[kMaxGN];
+#pragma unroll
+    for (int g = 0; g < kMaxGN; ++g) agv[g] = __shfl_sync(0xffffffffu, a_l, 8 * g);
+    constexpr int DW = WT == W_F16 ? 4 : 2;  // 32-bit words of a down chunk
+    uint32_t wdn[kMaxGN][CPT][DW];
+    float sdn[kMaxGN][CPT];
+#pragma unroll
+    for (int g = 0; g < kMaxGN; ++g)
+#pragma unroll
+      for (int cq = 0; cq < CPT; ++cq) {
+        if (WT == W_F16) {
+          const uint4 v = *reinterpret_cast<const uint4 *>(nd[g] + NL.down + coff[cq] * 16);
+          wdn[g][cq][0] = v.x;
+          wdn[g][cq][1] = v.y;
+          wdn[g][cq][DW - 2] = v.z;
+          wdn[g][cq][DW - 1] = v.w;
+          sdn[g][cq] = 1.f;
+        } else {
+          const uint2 v = *reinterpret_cast<const uint2 *>(nd[g] + NL.down + coff[cq] * 8);
+          wdn[g][cq][0] = v.x;
+          wdn[g][cq][DW - 1] = v.y;
+          sdn[g][cq] = __half2float(*reinterpret_cast<const __half *>(nd[g] + NL.sdown + (coff[cq] >> 1) * 2));
+        }
+      }
+#pragma unroll
+    for (int g = 0; g < kMaxGN; ++g) {
+      const float ag = agv[g];
+      if (g >= ng || ag == 0.f) continue;
 #pragma unroll
       for (int cq = 0; cq < CPT; ++cq) {
         if (WT == W_F16) {
           float w[8];
-          h8_to_f8(*reinterpret_cast<const uint4 *>(ndg + NL.down + coff[cq] * 16), w);
+          h8_to_f8(make_uint4(wdn[g][cq][0], wdn[g][cq][1], wdn[g][cq][DW - 2], wdn[g][cq][DW - 1]), w);
 #pragma unroll
           for (int e = 0; e < 8; ++e) y[cq][e] = fmaf(ag, w[e], y[cq][e]);
         } else {
-          const float sd = __half2float(*reinterpret_cast<const __half *>(ndg + NL.sdown + (coff[cq] >> 1) * 2));
-          const uint2 wq = *reinterpret_cast<const uint2 *>(ndg + NL.down + coff[cq] * 8);
+          const float sd = sdn[g][cq];
+          const uint2 wq = make_uint2(wdn[g][cq][0], wdn[g][cq][DW - 1]);
           const float as = ag * sd;
           // (q - 8) exactly, as the pairs (j, j + 4) of each 8-element word
           const __half2 off = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));
