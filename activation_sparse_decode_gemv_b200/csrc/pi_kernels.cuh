@@ -1,7 +1,7 @@
 // pi_kernels.cuh -- CUDA-core kernels of the predictor-gated sparse FFN
-// decode step (PowerInfer summary page: Summary, "lightweight per-layer
-// predictors" and "custom neuron-level sparse kernels"; Interesting ideas I4,
-// kernels that work directly on the rows of active neurons).
+// decode step (PowerInfer summary page: Summary, second paragraph, a small
+// predictor per layer and kernels specialised to single neurons; Interesting
+// ideas I4, kernels that work directly on the rows of active neurons).
 //
 // Per layer and token batch the chain is
 //   rmsnorm_kernel     (stacks only)  x fp32 -> u fp16

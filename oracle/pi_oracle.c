@@ -11,12 +11,13 @@
  * Language Model Serving with a Consumer-grade GPU", Elamur Research summary,
  * and the reboot-conseil overview):
  *   - per-layer predictor: a small model scores every FFN neuron and guesses
- *     which ones fire (Summary, "lightweight per-layer predictors"; Key points,
- *     Accuracy).  Here the predictor is the rank-r factorised scorer
- *     s = P2 (P1 u) + bias, and neuron i fires iff s_i > 0.
+ *     which ones fire (Summary, second paragraph; Key points, Accuracy).  Here
+ *     the predictor is the rank-r factorised scorer s = P2 (P1 u) + bias, and
+ *     neuron i fires iff s_i > 0.
  *   - neuron-aware sparse operator: only the rows of the active neurons are
- *     read and combined (Summary, "custom neuron-level sparse kernels skip the
- *     rest"; Interesting ideas I4, "operate directly on rows and columns").
+ *     read and combined, and the inactive ones are never touched (Summary,
+ *     second paragraph; Interesting ideas I4: kernels index the weight rows
+ *     and columns of the neurons themselves, with no sparse format).
  *     The result is exactly the dense FFN sum restricted to the chosen set:
  *         y_b = sum_{i in S_b} phi_i(u_b) * W2T_i
  *     with phi = ReLU(W1_i . u + b1_i) (OPT, Key points: ReLU) or
