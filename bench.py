@@ -38,16 +38,17 @@ import torch
 
 from activation_sparse_decode_gemv_b200 import inputs
 
-def kernels_per_step(cfg, B):
+def kernels_per_step(cfg, B, ids=False):
     """Launches of the library's kernels per decode step: batch 1 with fp16 /
     int4 weights runs as one persistent fused kernel; batches 16..32 with fp16
-    / int4 weights run six (token image, two tensor-core predictor GEMMs,
-    compaction, tensor-core up/gate and down GEMMs); otherwise five kernels
-    (predictor stage 1, stage 2, compaction, gather, reduction)."""
+    / int4 weights run five (token image, two tensor-core predictor GEMMs,
+    tensor-core up/gate and down GEMMs), plus the compaction when the call
+    asks for the id lists (``ids``); otherwise five kernels (predictor stage
+    1, stage 2, compaction, gather, reduction)."""
     if B == 1 and cfg.wtype != "f32" and cfg.r <= 1024 and cfg.d <= 8192:
         return 1
     if 16 <= B <= 32 and cfg.wtype != "f32" and (cfg.wtype != "int4g32" or cfg.d % 256 == 0):
-        return 6
+        return 6 if ids else 5
     return 5
 
 
@@ -454,7 +455,7 @@ def bench_ours(args, world, rank, local):
                                  if kernels_per_step(cfg, B) == 1 else None),
                      "algorithmic_bytes_per_launch": nbytes / args.steps,
                      "kernel": ("decode_fused_kernel (the whole step is one launch)" if kernels_per_step(cfg, B) == 1
-                                else "whole decode step (5 kernels)"),
+                                else f"whole decode step ({kernels_per_step(cfg, B)} kernels)"),
                      "peak_source": "measured" if "hbm_gbs" in peaks else "fallback"},
         "e2e": {"value": e2e_gbs, "unit": "GB/s", "h2d_bytes_per_step": int(toks[0].numel() * toks.element_size()),
                 "d2h_bytes_per_step": int(y.numel() * 4), "steps": n_e2e,
