@@ -108,3 +108,29 @@ def test_entry_points_reject_bad_arguments_without_launching(lib):
         assert lib.pi_workspace_size(arr, 1, 64, C.byref(C.c_size_t())) == pb.PI_ERR_UNSUPPORTED
     finally:
         lib.pi_ffn_destroy(h)
+
+
+def test_static_entry_and_status_calls_check_arguments_first(lib):
+    """pi_decode_ffn_static, pi_workspace_init and pi_get_device_status
+    reject bad arguments before any CUDA call (none is made on this host)."""
+    desc = _desc()
+    h = C.c_void_p()
+    assert lib.pi_ffn_create(C.byref(desc), C.byref(h)) == pb.PI_OK
+    try:
+        vp = C.c_void_p
+        st = lib.pi_decode_ffn_static
+        assert st(None, vp(0x100), vp(0x200), None, None, 0, None, None) == pb.PI_ERR_INVALID_ARG
+        assert st(h, None, vp(0x200), None, None, 0, None, None) == pb.PI_ERR_INVALID_ARG
+        assert st(h, vp(0x100), None, None, None, 0, None, None) == pb.PI_ERR_INVALID_ARG
+        assert st(h, vp(0x104), vp(0x200), None, None, 0, None, None) == pb.PI_ERR_MISALIGNED
+        assert st(h, vp(0x100), vp(0x208), None, None, 0, None, None) == pb.PI_ERR_MISALIGNED
+        assert st(h, vp(0x100), vp(0x200), vp(0x308), None, 0, None, None) == pb.PI_ERR_MISALIGNED
+        assert st(h, vp(0x100), vp(0x200), None, vp(0x404), 0, None, None) == pb.PI_ERR_MISALIGNED
+        assert st(h, vp(0x100), vp(0x200), None, None, 0, vp(0x502), None) == pb.PI_ERR_MISALIGNED
+        assert st(h, vp(0x100), vp(0x200), None, None, 8, None, None) == pb.PI_ERR_INVALID_ARG
+        assert lib.pi_workspace_init(None, 1024, None) == pb.PI_ERR_INVALID_ARG
+        assert lib.pi_workspace_init(vp(0x100), 0, None) == pb.PI_ERR_INVALID_ARG
+        assert lib.pi_get_device_status(None, None, C.byref(C.c_int())) == pb.PI_ERR_INVALID_ARG
+        assert lib.pi_get_device_status(vp(0x100), None, None) == pb.PI_ERR_INVALID_ARG
+    finally:
+        lib.pi_ffn_destroy(h)
