@@ -75,3 +75,22 @@ def test_profiled_traffic_parser(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "kernel_source_hash", lambda files=None: "other")
     assert bench.profiled_traffic("k.md") is None       # counters of other sources
     assert bench.profiled_traffic("missing.md") is None
+
+
+def test_reference_arm_line_on_cpu():
+    """bench.py --impl reference times the oracle on the host and prints one
+    JSON line with the contract's keys (small fp32 workload here)."""
+    import json
+    import subprocess
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config",
+                          "opt_tiny_f32", "--steps", "4", "--warmup", "3"], capture_output=True, text=True,
+                         timeout=300, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["higher_is_better"] is True
+    assert d["steps"] >= 1 and d["warmup"] == 3 and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
+    assert d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
