@@ -92,6 +92,39 @@ def _p(t: Optional[torch.Tensor]):
     return None if t is None else C.c_void_p(t.data_ptr())
 
 
+# The C ABI sees only pointers, so the binding checks what it cannot: each
+# tensor's dtype, size (at least the extent the header states) and
+# contiguity, then that all of them are CUDA tensors.  Null pointers and
+# everything the header validates are left to the library.
+def _need(t: Optional[torch.Tensor], what: str, dtype: torch.dtype, min_numel: int):
+    if t is None:
+        return
+    if t.dtype != dtype:
+        raise ValueError(f"{what}: dtype {t.dtype}, expected {dtype}")
+    if t.numel() < min_numel:
+        raise ValueError(f"{what}: {t.numel()} elements, the call needs at least {min_numel}")
+    if not t.is_contiguous():
+        raise ValueError(f"{what}: must be contiguous")
+
+
+def _on_device(**tensors: Optional[torch.Tensor]):
+    for what, t in tensors.items():
+        if t is not None and not t.is_cuda:
+            raise ValueError(f"{what}: must be a CUDA tensor")
+
+
+def _tokens(u: torch.Tensor, d: int, what: str) -> int:
+    """Batch size of a [B, d] token tensor."""
+    if u.dim() != 2 or u.shape[1] != d:
+        raise ValueError(f"{what}: shape {tuple(u.shape)}, expected [B, {d}]")
+    return u.shape[0]
+
+
+def _need_ws(ws: torch.Tensor):
+    if not ws.is_contiguous():
+        raise ValueError("workspace: must be contiguous")
+
+
 def _stream(stream=None):
     s = torch.cuda.current_stream() if stream is None else stream
     return C.c_void_p(s.cuda_stream)
@@ -109,6 +142,7 @@ class FfnLayer:
                                 _p(w_up), _p(w_gate), _p(w_down_t), _p(s_up), _p(s_gate), _p(s_down_t),
                                 _p(b_up), _p(p1), _p(p2), _p(p_bias))
         self.d, self.f, self.r, self.act, self.wtype = d, f, r, act, wtype
+        self.u_dtype = torch.float32 if wtype == "f32" else torch.float16  # FFN input u
         h = C.c_void_p()
         _check(lib().pi_ffn_create(C.byref(self.desc), C.byref(h)), "pi_ffn_create")
         self.handle = h
@@ -157,13 +191,26 @@ def _wsargs(ws: torch.Tensor):
 
 def pi_predict(layer: FfnLayer, u: torch.Tensor, idx: torch.Tensor, count: torch.Tensor, ws: torch.Tensor,
                stream=None):
-    B = u.shape[0]
+    """u [B, d]; idx int32 [B, f] (ascending ids, row b at b*f); count int32 [B]."""
+    B = _tokens(u, layer.d, "u")
+    _need(u, "u", layer.u_dtype, B * layer.d)
+    _need(idx, "idx", torch.int32, B * layer.f)
+    _need(count, "count", torch.int32, B)
+    _need_ws(ws)
+    _on_device(u=u, idx=idx, count=count, workspace=ws)
     _check(lib().pi_predict(layer.handle, _p(u), B, _p(idx), _p(count), *_wsargs(ws), _stream(stream)), "pi_predict")
 
 
 def pi_sparse_ffn(layer: FfnLayer, u: torch.Tensor, idx: torch.Tensor, count: torch.Tensor, y: torch.Tensor,
                   ws: torch.Tensor, flags: int = 0, stream=None):
-    B = u.shape[0]
+    """u [B, d]; idx int32 [B, f] and count int32 [B] (the sets); y fp32 [B, d]."""
+    B = _tokens(u, layer.d, "u")
+    _need(u, "u", layer.u_dtype, B * layer.d)
+    _need(idx, "idx", torch.int32, B * layer.f)
+    _need(count, "count", torch.int32, B)
+    _need(y, "y", torch.float32, B * layer.d)
+    _need_ws(ws)
+    _on_device(u=u, idx=idx, count=count, y=y, workspace=ws)
     _check(lib().pi_sparse_ffn(layer.handle, _p(u), B, _p(idx), _p(count), _p(y), int(flags), *_wsargs(ws),
                                _stream(stream)), "pi_sparse_ffn")
 
@@ -171,7 +218,14 @@ def pi_sparse_ffn(layer: FfnLayer, u: torch.Tensor, idx: torch.Tensor, count: to
 def pi_decode_ffn(layer: FfnLayer, u: torch.Tensor, y: torch.Tensor, ws: torch.Tensor,
                   idx: Optional[torch.Tensor] = None, count: Optional[torch.Tensor] = None, flags: int = 0,
                   stream=None):
-    B = u.shape[0]
+    """u [B, d]; y fp32 [B, d]; optional idx int32 [B, f] and count int32 [B]."""
+    B = _tokens(u, layer.d, "u")
+    _need(u, "u", layer.u_dtype, B * layer.d)
+    _need(y, "y", torch.float32, B * layer.d)
+    _need(idx, "idx", torch.int32, B * layer.f)
+    _need(count, "count", torch.int32, B)
+    _need_ws(ws)
+    _on_device(u=u, y=y, idx=idx, count=count, workspace=ws)
     _check(lib().pi_decode_ffn(layer.handle, _p(u), B, _p(y), _p(idx), _p(count), int(flags), *_wsargs(ws),
                                _stream(stream)), "pi_decode_ffn")
 
@@ -180,7 +234,14 @@ def pi_decode_ffn_static(layer: FfnLayer, u: torch.Tensor, y: torch.Tensor, idx:
                          count: Optional[torch.Tensor] = None, flags: int = 0,
                          dev_status: Optional[torch.Tensor] = None, stream=None):
     """Batch-1 decode step on the library's static device scratch (no workspace)."""
-    assert u.numel() == layer.d and y.numel() == layer.d, "pi_decode_ffn_static is batch 1"
+    if u.numel() != layer.d or y.numel() != layer.d:
+        raise ValueError("pi_decode_ffn_static is batch 1: u and y hold d elements")
+    _need(u, "u", layer.u_dtype, layer.d)
+    _need(y, "y", torch.float32, layer.d)
+    _need(idx, "idx", torch.int32, layer.f)
+    _need(count, "count", torch.int32, 1)
+    _need(dev_status, "dev_status", torch.int32, 1)
+    _on_device(u=u, y=y, idx=idx, count=count, dev_status=dev_status)
     _check(lib().pi_decode_ffn_static(layer.handle, _p(u), _p(y), _p(idx), _p(count), int(flags), _p(dev_status),
                                       _stream(stream)), "pi_decode_ffn_static")
 
@@ -188,8 +249,18 @@ def pi_decode_ffn_static(layer: FfnLayer, u: torch.Tensor, y: torch.Tensor, idx:
 def pi_decode_ffn_stack(layers: Sequence[FfnLayer], x: torch.Tensor, ws: torch.Tensor,
                         idx_trace: Optional[torch.Tensor] = None, count_trace: Optional[torch.Tensor] = None,
                         flags: int = 0, stream=None):
+    """x fp32 [B, d] (the residual, updated in place); optional idx_trace int32
+    [L, B, f_max] and count_trace int32 [L, B]."""
+    if not layers:
+        raise ValueError("pi_decode_ffn_stack needs at least one layer")
+    B = _tokens(x, layers[0].d, "x")
+    L, fmax = len(layers), max(l.f for l in layers)
+    _need(x, "x", torch.float32, B * layers[0].d)
+    _need(idx_trace, "idx_trace", torch.int32, L * B * fmax)
+    _need(count_trace, "count_trace", torch.int32, L * B)
+    _need_ws(ws)
+    _on_device(x=x, idx_trace=idx_trace, count_trace=count_trace, workspace=ws)
     arr = (C.c_void_p * len(layers))(*[l.handle for l in layers])
-    B = x.shape[0]
     _check(lib().pi_decode_ffn_stack(arr, len(layers), _p(x), B, _p(idx_trace), _p(count_trace), int(flags),
                                      *_wsargs(ws), _stream(stream)), "pi_decode_ffn_stack")
 
