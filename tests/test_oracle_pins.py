@@ -281,8 +281,8 @@ def test_single_neuron_closed_form_relu():
 def test_swiglu_closed_forms():
     """SiLU pins: with one-hot gate row e_k and up row e_m, phi = SiLU(u_k) u_m.
     Identities: SiLU(z) - SiLU(-z) = z; SiLU(0) = 0; SiLU(z) -> z for large z
-    and -> 0 for very negative z.  (exp itself comes from libm: parity of the
-    SiLU value beyond these identities is unpinned.)"""
+    and -> 0 for very negative z.  (The value itself is pinned against an
+    arbitrary-precision evaluation in the next test.)"""
     d, f = 8, 1
     Wg = np.zeros((f, d), np.float32); Wg[0, 2] = 1.0
     Wu = np.zeros((f, d), np.float32); Wu[0, 5] = 1.0
@@ -303,6 +303,37 @@ def test_swiglu_closed_forms():
     assert phi[0, 0] == 0.0
     assert abs(phi[1, 0] - 20.0) < 1e-6
     assert abs(phi[2, 0]) < 1e-20
+
+
+def test_silu_against_arbitrary_precision_definition():
+    """SiLU value pin: the oracle's SiLU(z) (a one-neuron SwiGLU layer with
+    one-hot gate and up rows, so phi = SiLU(z) * 1 exactly) against
+    z / (1 + e^-z) evaluated with Python's decimal module at 50 digits, an
+    exp independent of libm.  The oracle's double evaluation (exp, add,
+    divide) must agree to a few units in the last place."""
+    import decimal
+    decimal.getcontext().prec = 50
+    d, f = 8, 1
+    Wg = np.zeros((f, d), np.float32); Wg[0, 2] = 1.0
+    Wu = np.zeros((f, d), np.float32); Wu[0, 5] = 1.0
+    W2T = np.zeros((f, d), np.float32); W2T[0, 0] = 1.0
+    L = _manual_layer(Wu, W2T, np.zeros(f, np.float32), act="swiglu", Wg=Wg, wtype="f16")
+    # every fp16 value in [-20, 20] with a step of at least 1/64, plus both signs of tiny ones
+    zs = np.unique(np.concatenate([np.arange(-20.0, 20.0, 1.0 / 64), [2.0 ** -14, -2.0 ** -14, 2.0 ** -24]]))
+    zs = zs.astype(np.float16)
+    u = np.zeros((len(zs), d), np.float16)
+    u[:, 2] = zs
+    u[:, 5] = 1.0
+    phi = oracle.neuron_phi(L, u)[:, 0]
+    worst = 0.0
+    for z16, got in zip(zs, phi):
+        z = decimal.Decimal(float(z16))
+        exact = float(z / (1 + (-z).exp()))
+        if exact == 0.0:
+            assert got == 0.0
+            continue
+        worst = max(worst, abs(got - exact) / abs(exact))
+    assert worst <= 4 * 2.0 ** -53, worst
 
 
 def test_dense_matches_library_matmul():
