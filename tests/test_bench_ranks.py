@@ -52,3 +52,21 @@ def test_single_rank_is_identity():
     import bench
     gbs, t = bench.aggregate(2e9, 0.5, 1)
     assert gbs == pytest.approx(4.0) and t == 0.5
+
+
+def test_reference_arm_under_two_ranks():
+    """bench.py --impl reference under torchrun with 2 CPU ranks (gloo): rank 0
+    alone times the oracle and prints the one JSON line; the other rank exits
+    0 without work."""
+    import json
+    import subprocess
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), os.path.join(ROOT, "bench.py"),
+           "--impl", "reference", "--gpus", "2", "--config", "opt_tiny_f32", "--steps", "2", "--warmup", "3"]
+    out = subprocess.run(cmd, capture_output=True, text=True, timeout=300, cwd=ROOT,
+                         env={**os.environ, "CUDA_VISIBLE_DEVICES": ""})
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["steps"] >= 1
