@@ -15,7 +15,9 @@ from typing import List, Optional, Sequence
 import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libpi_ffn.so")
+# PI_FFN_LIB: another build of this library (the sanitizer test's host-
+# instrumented one); there is no non-CUDA implementation to fall back to
+LIB_PATH = os.environ.get("PI_FFN_LIB") or os.path.join(HERE, "libpi_ffn.so")
 
 PI_OK, PI_ERR_INVALID_ARG, PI_ERR_UNSUPPORTED, PI_ERR_MISALIGNED = 0, 1, 2, 3
 PI_ERR_CUDA, PI_ERR_TIMEOUT, PI_ERR_DEVICE_STATUS, PI_ERR_WORKSPACE = 4, 5, 6, 7

@@ -44,5 +44,21 @@ def build(force: bool = False, verbose: bool = False) -> str:
     return LIB
 
 
+def build_host_sanitized(out: str) -> str:
+    """The library with its HOST code built with AddressSanitizer and
+    UndefinedBehaviorSanitizer into ``out`` (device code as usual), for CPU
+    runs of the host-side tests; load it with the gcc sanitizer runtimes
+    preloaded.  (nvcc splits -Xcompiler values at commas, hence one flag per
+    sanitizer.)"""
+    flags = [f for f in FLAGS if f not in ("-O3", "-Xptxas", "-v")]
+    cmd = ([NVCC] + flags + ["-O1", "-g", "-Xcompiler", "-fsanitize=address", "-Xcompiler", "-fsanitize=undefined",
+                             "-Xcompiler", "-fno-omit-frame-pointer", "-o", out] + sources() + ["-lasan", "-lubsan"])
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if res.returncode != 0:
+        sys.stderr.write(res.stderr[-8000:])
+        raise RuntimeError("nvcc failed building the sanitized library")
+    return out
+
+
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))

@@ -24,5 +24,16 @@ def build(force: bool = False) -> str:
     return LIB
 
 
+def build_sanitized(out: str) -> str:
+    """The same oracle built with AddressSanitizer and UndefinedBehaviorSanitizer
+    (halting on the first report) into ``out``; load it with the gcc sanitizer
+    runtimes preloaded."""
+    cmd = ["gcc", "-std=c11", "-O1", "-g", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math",
+           "-fsanitize=address", "-fsanitize=undefined", "-fno-sanitize-recover=undefined",
+           "-fno-omit-frame-pointer", "-o", out, SRC, "-lm"]
+    subprocess.check_call(cmd)
+    return out
+
+
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv))
