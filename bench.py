@@ -70,7 +70,23 @@ def parse(argv=None):
     ap.add_argument("--json-out", default=None)
     ap.add_argument("--stack", action="store_true",
                     help="time pi_decode_ffn_stack through all layers of a stacked config (tokens/s)")
-    return ap.parse_args(argv)
+    ap.add_argument("--hot-mode", default="auto", choices=sorted(HOT_MODE_FLAGS),
+                    help="read the hot prefix densely, by index, or as the library decides (adds to --flags)")
+    ap.add_argument("--bias-norm", default=None, choices=["pred", "w1"],
+                    help="predictor bias scale of the generated layers (default: the config's)")
+    args = ap.parse_args(argv)
+    args.flags |= HOT_MODE_FLAGS[args.hot_mode]
+    return args
+
+
+# library flag bits (include/pi_ffn.h): PI_FFN_HOT_DENSE = 2, PI_FFN_HOT_INDEX = 4
+HOT_MODE_FLAGS = {"auto": 0, "dense": 2, "index": 4}
+
+
+def config_of(args) -> inputs.Config:
+    """The workload of --config, with the --bias-norm override."""
+    cfg = inputs.CONFIGS[args.config]
+    return cfg.scaled(bias_norm=args.bias_norm) if args.bias_norm else cfg
 
 
 # ----------------------------------------------------------------------------- distributed plumbing
@@ -269,7 +285,7 @@ def oracle_run(layer_host: inputs.LayerTensors, cfg, u_host: torch.Tensor, secon
 def bench_reference(args, world, rank):
     if rank != 0:
         return None
-    cfg = inputs.CONFIGS[args.config]
+    cfg = config_of(args)
     lt = inputs.make_layer(cfg, 0, seed=1000, device="cuda" if torch.cuda.is_available() else "cpu").to("cpu")
     toks = torch.stack([inputs.layer_input(cfg, inputs.make_tokens(cfg, t, args.batch, seed=1000))
                         for t in range(args.tokens)])
@@ -284,7 +300,7 @@ def bench_reference(args, world, rank):
             "us_per_layer": sec / n * 1e6, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic",
             "config": {"workload": f"{cfg.name} single FFN layer d={cfg.d} f={cfg.f} r={cfg.r} {cfg.wtype} "
-                                   f"batch {args.batch}", "batch": args.batch},
+                                   f"batch {args.batch}", "batch": args.batch, "bias_norm": cfg.bias_norm},
             "cpu_baseline": {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle",
                              "sample": f"{n} whole tokens of replica 0 (time-bounded at {args.ref_seconds:.0f} s)"},
             "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -296,7 +312,7 @@ def bench_ours(args, world, rank, local):
     assert torch.cuda.is_available(), "bench.py needs a CUDA device"
     pb.lib()
     dev = torch.device("cuda", local)
-    cfg = inputs.CONFIGS[args.config]
+    cfg = config_of(args)
     B, R, T = args.batch, args.replicas, args.tokens
     seed = 1000 + rank
     layers = [inputs.make_layer(cfg, r, seed=seed, device=dev) for r in range(R)]
@@ -452,7 +468,8 @@ def bench_ours(args, world, rank, local):
                                f"{cfg.wtype} weights, batch {B}, mean firing rate {cfg.mean_p}",
                    "batch": B, "d_model": cfg.d, "d_ffn": cfg.f, "rank": cfg.r, "replicas": R, "tokens": T,
                    "l2": f"{R} rotating seeded replicas ({sum(l.nbytes() for l in layers) / 1e9:.1f} GB) > L2",
-                   "bytes_per_step": nbytes / args.steps, "parallelism": f"replicas x{world}"},
+                   "bytes_per_step": nbytes / args.steps, "parallelism": f"replicas x{world}",
+                   "bias_norm": cfg.bias_norm, "hot_mode": args.hot_mode},
         "roofline": {"bound": "hbm", "achieved": per_gpu, "peak": peak, "unit": "GB/s", "frac": per_gpu / peak,
                      "traffic": (profiled_traffic(f"decode_fused_kernel_{cfg.name}_batch{B}.md")
                                  if kernels_per_step(cfg, B) == 1 else None),
@@ -484,7 +501,7 @@ def bench_stack(args, world, rank, local):
     assert torch.cuda.is_available(), "bench.py needs a CUDA device"
     pb.lib()
     dev = torch.device("cuda", local)
-    cfg = inputs.CONFIGS[args.config]
+    cfg = config_of(args)
     assert cfg.stacked, f"{cfg.name} is not a stacked config"
     B, L, T = args.batch, cfg.n_layers, args.tokens
     seed = 3000 + rank
@@ -558,7 +575,8 @@ def bench_stack(args, world, rank, local):
         "config": {"workload": f"{cfg.name}: {L}-layer FFN stack d={cfg.d} f={cfg.f} r={cfg.r} {cfg.act} "
                                f"{cfg.wtype} weights, batch {B}",
                    "batch": B, "layers": L, "tokens": T, "weights_gb": sum(l.nbytes() for l in layers) / 1e9,
-                   "bytes_per_step": nbytes / args.steps, "generation_s": gen_s},
+                   "bytes_per_step": nbytes / args.steps, "generation_s": gen_s,
+                   "bias_norm": cfg.bias_norm, "hot_mode": args.hot_mode},
         "roofline": {"bound": "hbm", "achieved": gbs / world, "peak": peak, "unit": "GB/s",
                      "frac": gbs / world / peak, "peak_source": "measured" if "hbm_gbs" in peaks else "fallback"},
         "clocks": clk.summary(),

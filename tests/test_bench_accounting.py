@@ -2,6 +2,7 @@
 against the published byte table of the workloads, the launch count it
 claims per step against the committed ncu launch lists, and the parser of
 profile summaries."""
+import dataclasses
 import os
 import sys
 
@@ -90,7 +91,19 @@ def test_reference_arm_line_on_cpu():
     assert len(lines) == 1
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["higher_is_better"] is True
+    assert d["config"]["bias_norm"] == "pred"
     assert d["steps"] >= 1 and d["warmup"] == 3 and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
     assert d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_cli_overrides():
+    a = bench.parse([])
+    assert a.flags == 0 and bench.config_of(a) is C["opt7b_f16"]
+    from activation_sparse_decode_gemv_b200 import binding as pb
+    a = bench.parse(["--hot-mode", "dense", "--flags", "1", "--bias-norm", "w1", "--config", "opt_tiny_f32"])
+    assert a.flags == pb.PI_FFN_ACCUMULATE | pb.PI_FFN_HOT_DENSE
+    assert bench.parse(["--hot-mode", "index"]).flags == pb.PI_FFN_HOT_INDEX
+    cfg = bench.config_of(a)
+    assert cfg.bias_norm == "w1" and dataclasses.replace(cfg, bias_norm="pred") == C["opt_tiny_f32"]
