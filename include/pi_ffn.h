@@ -120,21 +120,26 @@ pi_status pi_workspace_size(const pi_ffn_t *layers, int n_layers, int max_batch,
  * first use; kernels leave it reusable afterwards. */
 pi_status pi_workspace_init(void *ws, size_t ws_bytes, pi_stream_t stream);
 
-/* Predictor only (steps 1-2).  u: [B x d] (fp16, or fp32 for PI_W_F32).
+/* Predictor only (steps 1-2: the per-layer predictor of the summary page's
+ * Summary, second paragraph, sized per layer as in Interesting ideas I3).
+ * u: [B x d] (fp16, or fp32 for PI_W_F32).
  * idx: [B x f] int32, row b receives the ascending ids of token b's predicted
  * set in its first count[b] entries (the rest is left unspecified);
  * count: [B] int32. */
 pi_status pi_predict(pi_ffn_t h, const void *u, int B, int32_t *idx, int32_t *count, void *ws, size_t ws_bytes,
                      pi_stream_t stream);
 
-/* Sparse FFN over caller-supplied sets (steps 3-4).  idx/count as produced by
+/* Sparse FFN over caller-supplied sets (steps 3-4: kernels that read the
+ * rows and columns of the active neurons themselves, summary page,
+ * Interesting ideas I4).  idx/count as produced by
  * pi_predict (ids must lie in [0, f); a list is used as a set: order and
  * repeats do not matter; an out-of-range id is skipped and sets the device
  * status PI_ERR_DEVICE_STATUS).  y: [B x d] fp32 output.  flags: PI_FFN_*. */
 pi_status pi_sparse_ffn(pi_ffn_t h, const void *u, int B, const int32_t *idx, const int32_t *count, float *y,
                         unsigned flags, void *ws, size_t ws_bytes, pi_stream_t stream);
 
-/* Whole single-layer decode step (steps 1-4) from the FFN input u.  y: [B x d]
+/* Whole single-layer decode step (steps 1-4, the predictor-gated FFN of the
+ * summary page's Summary, second paragraph) from the FFN input u.  y: [B x d]
  * fp32.  idx/count: optional outputs as in pi_predict (NULL to skip).
  * Execution (the same for the predictor and sparse-FFN entry points where it
  * applies):
@@ -148,7 +153,9 @@ pi_status pi_decode_ffn(pi_ffn_t h, const void *u, int B, float *y, int32_t *idx
                         void *ws, size_t ws_bytes, pi_stream_t stream);
 
 /* Stacked decode through L layers of the same d_model (all fp16 or int4g32
- * weights): for each layer l, u = fp16(x / sqrt(mean(x^2) + 1e-6)) per token,
+ * weights).  The pages show no normalisation; the pre-FFN RMS norm below is
+ * this library's reading (the residual stream of a plain stack grows
+ * without bound): for each layer l, u = fp16(x / sqrt(mean(x^2) + 1e-6)) per token,
  * then steps 1-4, then the residual add x += y.  x: [B x d] fp32, in/out.
  * idx_trace: optional [L x B x f_max] int32 (layer l, token b at
  * (l*B + b)*f_max), count_trace: optional [L x B]. */
