@@ -24,15 +24,15 @@ PI_ERR_CUDA, PI_ERR_TIMEOUT, PI_ERR_DEVICE_STATUS, PI_ERR_WORKSPACE = 4, 5, 6, 7
 PI_ACT_RELU, PI_ACT_SWIGLU = 0, 1
 PI_W_F32, PI_W_F16, PI_W_INT4G32 = 0, 1, 2
 PI_FFN_ACCUMULATE, PI_FFN_HOT_DENSE, PI_FFN_HOT_INDEX = 1, 2, 4
-PI_STATIC_SCRATCH_BYTES = 4 * 1024 * 1024  # device scratch of pi_decode_ffn_static
+PI_STATIC_SCRATCH_BYTES = 16 * 1024 * 1024  # device scratch of pi_decode_ffn_static
 
 WTYPE = {"f32": PI_W_F32, "f16": PI_W_F16, "int4g32": PI_W_INT4G32}
 ACT = {"relu": PI_ACT_RELU, "swiglu": PI_ACT_SWIGLU}
 
 # every symbol the header declares
 EXPORTS = ("pi_ffn_create", "pi_ffn_destroy", "pi_workspace_size", "pi_workspace_init", "pi_predict",
-           "pi_sparse_ffn", "pi_decode_ffn", "pi_decode_ffn_stack", "pi_decode_ffn_static", "pi_get_device_status",
-           "pi_status_string")
+           "pi_sparse_ffn", "pi_decode_ffn", "pi_decode_ffn_stack", "pi_decode_ffn_static", "pi_debug_wait_fault",
+           "pi_get_device_status", "pi_status_string")
 
 
 class PiError(RuntimeError):
@@ -71,11 +71,13 @@ def lib() -> C.CDLL:
         L.pi_decode_ffn.argtypes = [vp, vp, i, vp, vp, vp, C.c_uint, vp, sz, vp]
         L.pi_decode_ffn_stack.argtypes = [C.POINTER(vp), i, vp, i, vp, vp, C.c_uint, vp, sz, vp]
         L.pi_decode_ffn_static.argtypes = [vp, vp, vp, vp, vp, C.c_uint, vp, vp]
+        L.pi_debug_wait_fault.argtypes = [i, C.c_uint]
         L.pi_get_device_status.argtypes = [vp, vp, C.POINTER(i)]
         L.pi_status_string.argtypes = [i]
         L.pi_status_string.restype = C.c_char_p
         for n in ("pi_ffn_create", "pi_workspace_size", "pi_workspace_init", "pi_predict", "pi_sparse_ffn",
-                  "pi_decode_ffn", "pi_decode_ffn_stack", "pi_decode_ffn_static", "pi_get_device_status"):
+                  "pi_decode_ffn", "pi_decode_ffn_stack", "pi_decode_ffn_static", "pi_debug_wait_fault",
+                  "pi_get_device_status"):
             getattr(L, n).restype = C.c_int
         _lib = L
     return _lib
@@ -265,6 +267,12 @@ def pi_decode_ffn_stack(layers: Sequence[FfnLayer], x: torch.Tensor, ws: torch.T
     arr = (C.c_void_p * len(layers))(*[l.handle for l in layers])
     _check(lib().pi_decode_ffn_stack(arr, len(layers), _p(x), B, _p(idx_trace), _p(count_trace), int(flags),
                                      *_wsargs(ws), _stream(stream)), "pi_decode_ffn_stack")
+
+
+def pi_debug_wait_fault(withhold_cta: int = -1, limit_us: int = 0):
+    """Test support: batch-1 fused launches withhold one CTA's slice of h and
+    wait at most ``limit_us`` (see the header); (-1, 0) restores normal runs."""
+    _check(lib().pi_debug_wait_fault(int(withhold_cta), int(limit_us)), "pi_debug_wait_fault")
 
 
 def pi_get_device_status(ws: torch.Tensor, stream=None) -> int:

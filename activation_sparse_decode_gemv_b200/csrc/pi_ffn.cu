@@ -22,6 +22,10 @@ struct pi_ffn {
   // TMA tensor maps of the tensor-core path (valid when tc_maps)
   bool tc_maps;
   CUtensorMap tm_p1, tm_p2, tm_up, tm_gate, tm_down, ts_up, ts_gate, ts_down;
+  // the batch-1 fused kernel's P2 tile map (valid when fx_ok, for fx_G CTAs)
+  bool fx_ok;
+  int fx_G, fx_M;
+  CUtensorMap tm_p2_fused;
 };
 
 namespace {
@@ -33,11 +37,15 @@ inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Workspace layout for a call at batch B on layers with the given maxima.
-// [0, 256): status region (int status, int union count, ...).
+// [0, 256): status region: int status, int union count, grid-barrier word,
+// and (at byte 64) the epoch of the fused kernel's tagged words.
+// fx_h / fx_part: the fused kernel's tagged exchange words (h, partials of y);
+// no other kernel writes them, so a stale word can never carry a current tag.
 struct WsLayout {
-  size_t h, u, mask, uwords, uprefix, ulist, partial, total;
+  size_t h, u, mask, uwords, uprefix, ulist, partial, fx_h, fx_part, total;
   int G;
 };
+constexpr size_t kEpochOffset = 64;
 
 int device_sm_count() {
   int dev = 0, n = 0;
@@ -64,6 +72,10 @@ WsLayout ws_layout(int dmax, int fmax, int rmax, int B, int G) {
   o = align_up(o + (size_t)fmax * 4, 256);
   L.partial = o;
   o = align_up(o + (size_t)G * B * dmax * 4, 256);
+  L.fx_h = o;
+  o = align_up(o + (size_t)rmax * 8, 256);
+  L.fx_part = o;
+  o = align_up(o + (size_t)G * dmax * 8, 256);
   L.total = o;
   L.G = G;
   return L;
@@ -166,6 +178,32 @@ bool build_tc_maps(pi_ffn *h) {
   return ok;
 }
 
+// The fused kernel's view of P2: the 4D tensor (k % 8, m, k / 8, c) of the
+// element k of neuron c + m G, for the G CTAs of one SM each and m < f / G,
+// so that one box {8, 32, r / 8, 1} brings a CTA's 32-row tile in the
+// K-interleaved order its ldmatrix reads.  Elements with m >= f / G read as
+// zero; the remaining f mod G rows are copied one per CTA.
+bool build_fused_map(pi_ffn *h) {
+  const pi_ffn_desc &D = h->d;
+  h->fx_ok = false;
+  const int G = device_sm_count();
+  if (G <= 0 || D.ptype != PI_W_F16 || D.rank % 16 || D.rank > 1024) return false;
+  h->fx_G = G;
+  h->fx_M = D.d_ffn / G;
+  if (h->fx_M == 0) return h->fx_ok = true;  // every row is a leftover row: no map
+  EncodeTiledFn enc = encoder();
+  if (!enc) return false;
+  const uint64_t r = (uint64_t)D.rank;
+  const cuuint64_t dims[4] = {8, (cuuint64_t)h->fx_M, r / 8, (cuuint64_t)G};
+  const cuuint64_t strides[3] = {(cuuint64_t)G * r * 2, 16, r * 2};
+  const cuuint32_t box[4] = {8, 32, (cuuint32_t)(r / 8), 1};
+  const cuuint32_t es[4] = {1, 1, 1, 1};
+  h->fx_ok = enc(&h->tm_p2_fused, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void *>(D.p2), dims, strides, box,
+                 es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return h->fx_ok;
+}
+
 constexpr int kTcMinBatch = 16;
 
 struct Ws {
@@ -183,6 +221,9 @@ struct Ws {
   int32_t *uprefix() const { return reinterpret_cast<int32_t *>(base + L.uprefix); }
   int32_t *ulist() const { return reinterpret_cast<int32_t *>(base + L.ulist); }
   float *partial() const { return reinterpret_cast<float *>(base + L.partial); }
+  unsigned *epoch() const { return reinterpret_cast<unsigned *>(base + kEpochOffset); }
+  unsigned long long *fx_h() const { return reinterpret_cast<unsigned long long *>(base + L.fx_h); }
+  unsigned long long *fx_part() const { return reinterpret_cast<unsigned long long *>(base + L.fx_part); }
   unsigned char *uimg() const { return reinterpret_cast<unsigned char *>(tc + T.uimg); }
   unsigned char *uimg_perm() const { return reinterpret_cast<unsigned char *>(tc + T.uimg_perm); }
   unsigned char *himg_hi() const { return reinterpret_cast<unsigned char *>(tc + T.himg_hi); }
@@ -568,6 +609,14 @@ pi_status run_ffn_tc(const pi_ffn *h, const void *u, int B, float *out, int accu
 // ---------------------------------------------------------------- fused batch-1 path
 namespace F = pi::fused;
 
+// Test support (pi_debug_wait_fault): a CTA that withholds its slice of h and
+// a shorter limit for every bounded wait of the fused kernel.
+struct WaitFault {
+  int withhold = -1;
+  unsigned long long limit_ns = 0;  // 0: the kernel's default
+};
+WaitFault g_wait_fault;
+
 template <int WT, int ACT, int CPT>
 cudaError_t fused_launch(const F::Args &a, int G, cudaStream_t st) {
   static bool attr_set = false;
@@ -587,26 +636,17 @@ cudaError_t fused_launch(const F::Args &a, int G, cudaStream_t st) {
   cfg.blockDim = dim3(F::kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  // cooperative (all CTAs co-resident for the grid barriers) and, where the
-  // runtime accepts the pair, programmatic dependent launch
-  static int pdl_ok = -1;
-  cudaLaunchAttribute at[2];
-  at[0].id = cudaLaunchAttributeCooperative;
-  at[0].val.cooperative = 1;
-  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  at[1].val.programmaticStreamSerializationAllowed = 1;
+  // Programmatic dependent launch, and no cooperative attribute: a
+  // cooperative grid is only scheduled once every SM is free, while here the
+  // CTAs of the next launch take the SMs of this launch's CTAs as they leave
+  // and start streaming weights during its reduction.  The grid is one CTA per
+  // SM and every wait for another CTA is bounded, so CTAs that cannot all be
+  // resident (another kernel holding SMs for longer than the limit) end in
+  // PI_ERR_TIMEOUT, never in a hang.
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
-  if (pdl_ok != 0) {
-    cfg.numAttrs = 2;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, F::decode_fused_kernel<WT, ACT, CPT>, a);
-    if (e == cudaSuccess) {
-      pdl_ok = 1;
-      return e;
-    }
-    if (pdl_ok == 1) return e;
-    cudaGetLastError();
-    pdl_ok = 0;
-  }
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, F::decode_fused_kernel<WT, ACT, CPT>, a);
 }
@@ -615,7 +655,8 @@ cudaError_t fused_launch(const F::Args &a, int G, cudaStream_t st) {
 // fp16 predictor of rank <= 1024, and one neuron's rows fitting one slot.
 bool fused_ok(const pi_ffn *h, int B, int G) {
   const pi_ffn_desc &D = h->d;
-  if (B != 1 || D.ptype != PI_W_F16 || D.rank > F::kMaxR || G > 320) return false;
+  if (B != 1 || D.ptype != PI_W_F16 || D.rank > F::kMaxR || D.rank % 16 || G > 320) return false;
+  if (!h->fx_ok || h->fx_G != G) return false;
   if (D.wtype == PI_W_F16) {
     if (D.d_model > 8192) return false;
   } else if (D.wtype == PI_W_INT4G32) {
@@ -635,6 +676,8 @@ pi_status run_fused(const pi_ffn *h, const void *in, float *out, int stack, int 
                     int32_t *count, unsigned flags, const Ws &w, cudaStream_t st) {
   const pi_ffn_desc &D = h->d;
   F::Args a{};
+  a.tm_p2 = h->tm_p2_fused;
+  a.p2_main = h->fx_M;
   a.w_up = D.w_up;
   a.w_gate = D.w_gate;
   a.w_down_t = D.w_down_t;
@@ -653,24 +696,27 @@ pi_status run_fused(const pi_ffn *h, const void *in, float *out, int stack, int 
   a.stack = stack;
   a.accumulate = accumulate;
   a.H = want_dense(h, 1, flags) ? h->H : 0;
-  a.h = w.h();
-  a.partial = w.partial();
+  a.hx = w.fx_h();
+  a.px = w.fx_part();
+  a.epoch = w.epoch();
   a.mask32 = w.mask();
   a.bar = w.grid_bar();
   a.status = w.status();
   a.idx = idx;
   a.count = count;
+  a.wait_ns = g_wait_fault.limit_ns ? g_wait_fault.limit_ns : F::kWaitNs;
+  a.withhold = g_wait_fault.withhold;
   cudaError_t e;
   const bool relu = D.act == PI_ACT_RELU;
   const int G = w.L.G;
   if (D.wtype == PI_W_F16) {
-    if (D.d_model <= 2 * F::kConsumers * 8)
-      e = relu ? fused_launch<pi::W_F16, pi::ACT_RELU, 2>(a, G, st) : fused_launch<pi::W_F16, pi::ACT_SWIGLU, 2>(a, G, st);
+    if (D.d_model <= F::kConsumers * 8)
+      e = relu ? fused_launch<pi::W_F16, pi::ACT_RELU, 1>(a, G, st) : fused_launch<pi::W_F16, pi::ACT_SWIGLU, 1>(a, G, st);
     else
-      e = relu ? fused_launch<pi::W_F16, pi::ACT_RELU, 4>(a, G, st) : fused_launch<pi::W_F16, pi::ACT_SWIGLU, 4>(a, G, st);
+      e = relu ? fused_launch<pi::W_F16, pi::ACT_RELU, 2>(a, G, st) : fused_launch<pi::W_F16, pi::ACT_SWIGLU, 2>(a, G, st);
   } else {
-    e = relu ? fused_launch<pi::W_INT4, pi::ACT_RELU, 2>(a, G, st)
-             : fused_launch<pi::W_INT4, pi::ACT_SWIGLU, 2>(a, G, st);
+    e = relu ? fused_launch<pi::W_INT4, pi::ACT_RELU, 1>(a, G, st)
+             : fused_launch<pi::W_INT4, pi::ACT_SWIGLU, 1>(a, G, st);
   }
   return e == cudaSuccess ? PI_OK : PI_ERR_CUDA;
 }
@@ -695,21 +741,50 @@ namespace {
 
 constexpr int kMaxStaticDevices = 64;
 std::mutex g_static_mu;
-void *g_static_ptr[kMaxStaticDevices];
+struct StaticEntry {
+  void *ctx = nullptr;  // context the address belongs to
+  void *ptr = nullptr;
+};
+StaticEntry g_static[kMaxStaticDevices];
 
-// Device address of the scratch array on the current device, looked up once
-// per device (with that device current) and cached.
+// The current context (cuCtxGetCurrent through the runtime's driver entry
+// point), so that a cached address is reused only inside the context it was
+// looked up in: a device reset or a new primary context reloads the module,
+// and the array can move.
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+void *current_context() {
+  static CtxGetCurrentFn fn = []() -> CtxGetCurrentFn {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !p) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    return reinterpret_cast<CtxGetCurrentFn>(p);
+  }();
+  CUcontext c = nullptr;
+  if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
+// Device address of the scratch array on the current device, looked up with
+// that device current the first time a context uses it, then cached for the
+// context.
 pi_status static_scratch(void **out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return PI_ERR_CUDA;
   if (dev < 0 || dev >= kMaxStaticDevices) return PI_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_static_mu);
-  if (!g_static_ptr[dev]) {
+  void *ctx = current_context();
+  StaticEntry &e = g_static[dev];
+  if (!e.ptr || !ctx || e.ctx != ctx) {
     void *p = nullptr;
     if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return PI_ERR_CUDA;
-    g_static_ptr[dev] = p;
+    e.ptr = p;
+    e.ctx = current_context();  // the lookup makes the primary context current if none was
   }
-  *out = g_static_ptr[dev];
+  *out = e.ptr;
   return PI_OK;
 }
 
@@ -747,6 +822,7 @@ pi_status pi_ffn_create(const pi_ffn_desc *desc, pi_ffn_t *out) {
   h->H = D.hot_prefix & ~31;
   h->nwords = (D.d_ffn + 31) / 32;
   h->tc_maps = build_tc_maps(h);
+  build_fused_map(h);
   *out = h;
   return PI_OK;
 }
@@ -899,6 +975,14 @@ pi_status pi_decode_ffn_static(pi_ffn_t h, const void *u, float *y, int32_t *idx
   }
   if (s != PI_OK) return s;
   if (dev_status) PI_CUDA(cudaMemcpyAsync(dev_status, base, sizeof(int), cudaMemcpyDeviceToDevice, st));
+  return PI_OK;
+}
+
+pi_status pi_debug_wait_fault(int withhold_cta, unsigned limit_us) {
+  if (withhold_cta < -1) return PI_ERR_INVALID_ARG;
+  if (withhold_cta >= 0 && limit_us == 0) return PI_ERR_INVALID_ARG;
+  g_wait_fault.withhold = withhold_cta;
+  g_wait_fault.limit_ns = (unsigned long long)limit_us * 1000ull;
   return PI_OK;
 }
 

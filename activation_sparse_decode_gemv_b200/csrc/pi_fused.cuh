@@ -4,33 +4,48 @@
 // read the rows of the active neurons directly).
 //
 // Grid: one CTA per SM, launched cooperatively (all CTAs co-resident).
-// Block: 8 consumer warps + 1 producer warp.  The producer streams work items
-// into a ring of 3 x 64 KB shared-memory slots with cp.async.bulk (TMA bulk
-// copies) and mbarrier transaction counts; consumers process the slots in
-// order:
-//   P1 item     up to 8 rows of P1 owned by this CTA -> its slice of h = P1 u
-//               (then a grid-wide barrier publishes all of h)
-//   P2 tile     32 predictor rows -> s = P2 h + bias, fire iff s > 0.  Warps
-//               record the fired bits with shared-memory atomics and release
-//               the slot without a block barrier.
+// Block: 16 consumer warps + 1 producer warp.  The producer streams work items
+// into a ring of 3 shared-memory slots with cp.async.bulk (TMA bulk copies)
+// and mbarrier transaction counts; consumers process the slots in order:
+//   P1 item     up to 8 rows of P1 owned by this CTA -> its slice of h = P1 u,
+//               published to every CTA as tagged words (below)
+//   P2 tile     32 predictor rows -> s = P2 h + bias, fire iff s > 0.  The
+//               dot products run on the tensor cores (mma.sync m16n8k16):
+//               A = the tile's rows, B = h split into h_hi = fp16(h) and
+//               h_lo = fp16(h - h_hi) as the first two of the 8 columns, so
+//               s = D[:,0] + D[:,1] carries h to about 22 bits.  Each warp
+//               takes one eighth of the rank; the last warp to finish a tile
+//               adds the eight partial sums in warp order and sets the fired
+//               bits, so no block barrier is needed per tile.
 //   GATHER      up (+gate) and down rows of 1-4 neurons: dot with u,
 //               activation, then y += a * W2T_i in per-thread registers
 //   DONE        end of the stream
 // The producer "harvests" a tile when its slot's empty barrier completes
 // (every consumer warp is done with it), appends the fired ids to its list
-// and issues their gather rows; it keeps issuing P2 tiles meanwhile, and it
-// prefetches tiles while the consumers wait on the h barrier.  Neurons are
-// dealt round robin to the CTAs (neuron i to CTA i mod G), so every CTA gets
-// the same mix of hot and cold neurons; CTA c's k-th tile holds its own
-// neurons c + (32k + q) G, q < 32.  In dense hot-prefix mode the rows of a
-// tile's prefix neurons are issued right after the tile, without waiting
-// for its bits.
-// After the stream every CTA writes its fp32 partial of y; a second grid
-// barrier; each CTA then sums a column slice over all partials in CTA order
-// (deterministic, no atomics) and writes y (or adds it to the residual x).
+// and issues their gather rows; it keeps issuing P2 tiles meanwhile.  At the
+// start it also asks L2 for all of this CTA's P2 rows (bulk L2 prefetch), so
+// HBM keeps streaming the predictor while the ring is full and h is not yet
+// known.  Neurons are dealt round robin to the CTAs (neuron i to CTA i mod G),
+// so every CTA gets the same mix of hot and cold neurons; CTA c's k-th tile
+// holds its own neurons c + (32k + q) G, q < 32.  In dense hot-prefix mode the
+// rows of a tile's prefix neurons are issued right after the tile, without
+// waiting for its bits.
+//
+// Cross-CTA exchanges carry their own readiness: every value goes out as one
+// 64-bit word (value bits, tag), stored and loaded with single-copy-atomic
+// relaxed gpu-scope accesses.  The tag is the launch's epoch + 1; the epoch
+// lives in the workspace, every CTA reads it after griddepcontrol.wait, and
+// CTA 0 advances it once its reduction has seen every CTA's partial (so every
+// CTA has read it).  A reader polls until the tag matches, so publishing h or
+// a partial of y costs one L2 round trip and no grid barrier.  After the
+// stream every CTA publishes its fp32 partial of y; each CTA then sums a
+// column slice over all partials in CTA order (deterministic, no atomics) and
+// writes y (or adds it to the residual x).
 // Every wait is bounded (about 2 s); on expiry the kernel records
 // PI_ERR_TIMEOUT in the workspace status word and completes.
 #pragma once
+
+#include <cuda.h>
 
 #include <cstddef>
 
@@ -39,17 +54,22 @@
 namespace pi {
 namespace fused {
 
-constexpr int kConsumerWarps = 8;
+constexpr int kConsumerWarps = 16;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kThreads = kConsumers + 32;
 constexpr int kSlots = 3;
-constexpr int kSlotBytes = 65536;
 constexpr int kTN = 32;                      // neurons per predictor tile
+constexpr int kMaxR = 1024;                  // predictor rank
+// a slot holds one item: a predictor tile (32 rows of the rank, K-interleaved,
+// plus the CTA's leftover row), up to 8 rows of P1, or the rows of 1-4 neurons
+constexpr int kSlotBytes = (kTN + 1) * 2 * kMaxR;
 constexpr int kMaxGN = 4;                    // neurons per gather item
 constexpr int kMaxOwnTiles = 32;             // neurons per CTA <= 32 * 32
 constexpr int kActCap = kMaxOwnTiles * kTN;  // capacity of the active-id list
-constexpr int kMaxR = 1024;                  // predictor rank
 constexpr int kMaxP1Rows = 8;                // P1 rows per item
+constexpr int kMaxKs = kMaxR / 16 / kConsumerWarps;  // k16 steps of the rank per consumer warp
+constexpr int kRedCols = 64;                 // columns of y each reducing CTA sums
+constexpr int kRedBatch = 10;                // partials polled per batch by one reducing thread
 constexpr unsigned long long kWaitNs = 2000000000ull;
 
 enum ItemType : int { IT_P1 = 0, IT_P2 = 1, IT_GATHER = 2, IT_DONE = 3 };
@@ -65,25 +85,34 @@ struct Smem {
   unsigned long long full[kSlots];
   unsigned long long empty[kSlots];
   unsigned tbits[kSlots];              // fired bits of the tile in a slot
+  int tdone[kSlots];                   // consumer warps done with the tile in a slot
   unsigned own_bits[kMaxOwnTiles];     // fired bits of this CTA's tiles
   int act[kActCap];                    // fired ids (index mode), producer-owned
   int tile_item[kMaxOwnTiles];         // item number each own tile was issued as
   float own_pbias[kMaxOwnTiles][kTN];  // predictor bias of this CTA's neurons
   float own_bup[kMaxOwnTiles][kTN];    // ReLU bias b1 of this CTA's neurons
-  alignas(16) float h_s[kMaxR];  // written with 16-byte vector stores
+  float h_s[kMaxR];                    // h, gathered from all CTAs
+  float spart[kSlots][kConsumerWarps][kTN];  // per-warp partial scores of a tile
   float red[2][kConsumerWarps][2 * kMaxGN];
   double dred[kConsumerWarps];
-  float fin[kConsumerWarps][33];
+  float fin[kConsumers / (kRedCols / 2)][kRedCols + 1];
   int iscan[kConsumerWarps];
   volatile int abort_flag;
 };
 
 static_assert(offsetof(Smem, ring) == 0, "ring slots must start the shared block");
 static_assert(kSlotBytes % 16 == 0, "bulk copies need 16-byte aligned slots");
-static_assert(offsetof(Smem, h_s) % 16 == 0, "h_s is accessed with 16-byte vectors");
+static_assert(kSlotBytes % 128 == 0, "tensor copies need 128-byte aligned slots");
 static_assert(sizeof(Smem) <= 227 * 1024, "shared memory per block");
+static_assert(kConsumers * 2 * kRedBatch * 4 <= kSlots * kSlotBytes, "reduction stage fits the ring");
 
 struct Args {
+  // P2 as the 4D tensor (k % 8, m, k / 8, c) of neuron c + m G's element k,
+  // m < f / G: one box {8, 32, r / 8, 1} is the 32 rows of a CTA's tile,
+  // stored K-interleaved ([k / 8][row][k % 8], 16 bytes per row and chunk),
+  // which ldmatrix reads without bank conflicts; rows past f / G read as 0
+  CUtensorMap tm_p2;
+  int p2_main;     // f / G (0: no main rows, and tm_p2 is not used)
   const void *w_up, *w_gate, *w_down_t;
   const __half *s_up, *s_gate, *s_down_t;
   const float *b_up;
@@ -95,13 +124,16 @@ struct Args {
   int stack;       // input is the residual x: RMS-normalise it, and add y into it
   int accumulate;  // y += (non-stack)
   int H;           // dense hot-prefix neurons [0, H); 0 = index mode
-  float *h;        // workspace [r]
-  float *partial;  // workspace [G x d]
+  unsigned long long *hx;  // workspace [r] tagged h
+  unsigned long long *px;  // workspace [G x d] tagged partials of y
+  unsigned *epoch;         // workspace launch counter of the tags
   unsigned *mask32;  // workspace [ceil(f/32)] fired bits of neurons 32w..32w+31, when idx or count != nullptr
-  unsigned *bar;     // workspace grid-barrier word
+  unsigned *bar;     // workspace grid-barrier word (id lists only)
   int *status;
   int32_t *idx;    // optional ascending active ids [f]
   int32_t *count;  // optional [1]
+  unsigned long long wait_ns;  // limit of every bounded wait
+  int withhold;    // CTA that does not publish its slice of h (-1: none); exercises the bounded waits
 };
 
 // ---------------------------------------------------------------- PTX helpers
@@ -120,17 +152,6 @@ PI_DEV void mbar_arrive_tx(unsigned long long *b, unsigned tx) {
 PI_DEV void mbar_arrive(unsigned long long *b) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
 }
-// try_wait with a suspend-time hint: the thread is parked until the phase
-// completes or the hint (ns) elapses, instead of spinning on the barrier
-PI_DEV bool mbar_try(unsigned long long *b, unsigned parity, unsigned hint_ns) {
-  unsigned ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(b)), "r"(parity), "r"(hint_ns)
-      : "memory");
-  return ok != 0;
-}
 PI_DEV bool mbar_test(unsigned long long *b, unsigned parity) {
   unsigned ok;
   asm volatile(
@@ -140,22 +161,27 @@ PI_DEV bool mbar_test(unsigned long long *b, unsigned parity) {
       : "memory");
   return ok != 0;
 }
-// bounded wait; false on timeout (status recorded).  The fast path (phase
-// already complete) is inline, the suspending loop is out of line to keep
-// the consumer loop small in the instruction cache.
-__device__ __noinline__ bool mbar_wait_slow(unsigned long long *b, unsigned parity, int *status) {
+// bounded wait; false on timeout (status recorded).  It polls with
+// test_wait and a short back-off: a thread parked by try_wait's suspend hint
+// was measured to resume up to ~2 us after the phase completed, which delayed
+// the producer's next copy by as much.  The fast path (phase already
+// complete) is inline, the polling loop is out of line to keep the consumer
+// loop small in the instruction cache.
+__device__ __noinline__ bool mbar_wait_slow(unsigned long long *b, unsigned parity, int *status,
+                                            unsigned long long limit) {
   const unsigned long long t0 = globaltimer();
   for (;;) {
-    if (mbar_try(b, parity, 20000u)) return true;
-    if (globaltimer() - t0 > kWaitNs) {
+    if (mbar_test(b, parity)) return true;
+    if (globaltimer() - t0 > limit) {
       set_status(status, kStatusTimeout);
       return false;
     }
+    __nanosleep(20);
   }
 }
-PI_DEV bool mbar_wait(unsigned long long *b, unsigned parity, int *status) {
+PI_DEV bool mbar_wait(unsigned long long *b, unsigned parity, int *status, unsigned long long limit) {
   if (mbar_test(b, parity)) return true;
-  return mbar_wait_slow(b, parity, status);
+  return mbar_wait_slow(b, parity, status, limit);
 }
 PI_DEV void bulk_g2s(void *dst, const void *src, unsigned bytes, unsigned long long *bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
@@ -163,31 +189,91 @@ PI_DEV void bulk_g2s(void *dst, const void *src, unsigned bytes, unsigned long l
                "l"(src), "r"(bytes), "r"(smem_u32(bar))
                : "memory");
 }
+// 4D TMA box load at element coordinates (x0, x1, x2, x3) of a tensor map
+// (a kernel parameter); elements outside the tensor read as zero
+PI_DEV void tma_load_4d(void *dst, const CUtensorMap *tm, int x0, int x1, int x2, int x3, unsigned long long *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], "
+      "[%6];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<unsigned long long>(tm)), "r"(x0), "r"(x1), "r"(x2), "r"(x3), "r"(smem_u32(bar))
+      : "memory");
+}
 PI_DEV void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kConsumers) : "memory"); }
 PI_DEV unsigned ld_acquire(const unsigned *p) {
   unsigned v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
-PI_DEV float ld_cg(const float *p) { return __ldcg(p); }
+PI_DEV unsigned ld_relaxed_u32(const unsigned *p) {
+  unsigned v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+PI_DEV void st_relaxed_u32(unsigned *p, unsigned v) {
+  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
 
-// Grid-wide barrier, one thread per CTA.  Every CTA adds 1 except CTA 0,
-// which adds 2^31 - (G - 1): the word's top bit flips exactly when all G
-// have arrived, and the low bits return to their previous value, so the
-// word never needs resetting between barriers or launches.
-PI_DEV bool grid_barrier(unsigned *bar, int G, int c, int *status) {
+// ---------------------------------------------------------------- tagged words
+// (value, tag) as one 64-bit word: low half the value's bits, high half the tag
+PI_DEV unsigned long long tagged(float v, unsigned tag) {
+  return ((unsigned long long)tag << 32) | (unsigned long long)__float_as_uint(v);
+}
+PI_DEV float tagged_value(unsigned long long w) { return __uint_as_float((unsigned)(w & 0xffffffffull)); }
+PI_DEV bool tag_is(unsigned long long w, unsigned tag) { return (unsigned)(w >> 32) == tag; }
+PI_DEV void st_tagged(unsigned long long *p, unsigned long long w) {
+  asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
+}
+PI_DEV void st_tagged2(unsigned long long *p, unsigned long long w0, unsigned long long w1) {
+  asm volatile("st.relaxed.gpu.global.v2.b64 [%0], {%1, %2};" ::"l"(p), "l"(w0), "l"(w1) : "memory");
+}
+// two consecutive tagged words (16-byte aligned); each is its own
+// single-copy-atomic 64-bit access
+PI_DEV void ld_tagged2(const unsigned long long *p, unsigned long long &w0, unsigned long long &w1) {
+  asm volatile("ld.relaxed.gpu.global.v2.b64 {%0, %1}, [%2];" : "=l"(w0), "=l"(w1) : "l"(p) : "memory");
+}
+
+// Grid-wide barrier, one thread per CTA (used only when the call asks for
+// the global id list).  Every CTA adds 1 except CTA 0, which adds
+// 2^31 - (G - 1): the word's top bit flips exactly when all G have arrived,
+// and the low bits return to their previous value, so the word never needs
+// resetting between barriers or launches.
+PI_DEV bool grid_barrier(unsigned *bar, int G, int c, int *status, unsigned long long limit) {
   const unsigned inc = (c == 0) ? (0x80000000u - (unsigned)(G - 1)) : 1u;
   __threadfence();
   const unsigned old = atomicAdd(bar, inc);
   const unsigned long long t0 = globaltimer();
   for (;;) {
     if (((ld_acquire(bar) ^ old) & 0x80000000u) != 0u) return true;
-    if (globaltimer() - t0 > kWaitNs) {
+    if (globaltimer() - t0 > limit) {
       set_status(status, kStatusTimeout);
       return false;
     }
     __nanosleep(64);
   }
+}
+
+// ---------------------------------------------------------------- tensor-core helpers
+PI_DEV void ldmatrix_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+// D += A B with A 16x16 fp16 (row-major fragments), B 16x8 fp16, D fp32
+PI_DEV void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// fp16 pair (lo element first) of the high or low part of two fp32 values
+PI_DEV uint32_t h_part_pair(float x0, float x1, int lo) {
+  const __half a0 = __float2half_rn(x0), a1 = __float2half_rn(x1);
+  __half v0 = a0, v1 = a1;
+  if (lo) {
+    v0 = __float2half_rn(x0 - __half2float(a0));
+    v1 = __float2half_rn(x1 - __half2float(a1));
+  }
+  return (uint32_t)__half_as_ushort(v0) | ((uint32_t)__half_as_ushort(v1) << 16);
 }
 
 // ---------------------------------------------------------------- element types
@@ -201,32 +287,6 @@ template <> struct Cols<W_INT4> {
   static constexpr int EC = 16;
 };
 
-// dot of 8 fp16 weights with 8 fp32 values as two independent chains
-PI_DEV float dot8_h2(const uint4 &w, const float *u) {
-  const __half2 *hp = reinterpret_cast<const __half2 *>(&w);
-  const float2 a0 = __half22float2(hp[0]), a1 = __half22float2(hp[1]);
-  const float2 a2 = __half22float2(hp[2]), a3 = __half22float2(hp[3]);
-  float x = a0.x * u[0], y = a0.y * u[1];
-  x = fmaf(a1.x, u[2], x);
-  y = fmaf(a1.y, u[3], y);
-  x = fmaf(a2.x, u[4], x);
-  y = fmaf(a2.y, u[5], y);
-  x = fmaf(a3.x, u[6], x);
-  y = fmaf(a3.y, u[7], y);
-  return x + y;
-}
-// 16 int4 values (one 8-byte word pair) times u, without the group scale,
-// as two independent chains
-PI_DEV float dot16_q(uint2 w, const float *u) {
-  float x = 0.f, y = 0.f;
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    x = fmaf((float)((int)((w.x >> (4 * k)) & 15u) - 8), u[k], x);
-    y = fmaf((float)((int)((w.y >> (4 * k)) & 15u) - 8), u[8 + k], y);
-  }
-  return x + y;
-}
-
 // 8 fp16 weights times 8 fp16 inputs (16 B each), accumulated into two fp32
 // chains with the mixed-precision FMA: the product of two fp16 values is exact
 // in fp32, so each step equals fmaf((float)w, (float)u, acc) bit for bit
@@ -238,27 +298,6 @@ PI_DEV void dot8_mixed(const uint4 &w, const uint4 &u, float &x, float &y) {
         " fma.rn.f32.f16 %0, al, bl, %0;\n fma.rn.f32.f16 %1, ah, bh, %1;\n}\n"
         : "+f"(x), "+f"(y)
         : "r"(ws[k]), "r"(us[k]));
-}
-// the 8 int4 codes of one 32-bit word (element 2k = low nibble of byte k) as
-// four fp16 pairs (q - 8): 0x6400 | q is the fp16 value 1024 + q, and
-// subtracting 1032 is exact
-PI_DEV void q8_to_h2(uint32_t w, uint32_t out[4]) {
-  const __half2 off = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const uint32_t t = w >> (8 * k);
-    const uint32_t hb = (t & 0xFu) | ((t & 0xF0u) << 12) | 0x64006400u;
-    const __half2 v = __hsub2(*reinterpret_cast<const __half2 *>(&hb), off);
-    out[k] = *reinterpret_cast<const uint32_t *>(&v);
-  }
-}
-// 16 int4 codes (q - 8) times 16 fp16 inputs, without the group scale
-PI_DEV void dot16_q_mixed(const uint2 &w, const uint4 &u0, const uint4 &u1, float &x, float &y) {
-  uint32_t q[8];
-  q8_to_h2(w.x, q);
-  q8_to_h2(w.y, q + 4);
-  dot8_mixed(make_uint4(q[0], q[1], q[2], q[3]), u0, x, y);
-  dot8_mixed(make_uint4(q[4], q[5], q[6], q[7]), u1, x, y);
 }
 
 // the 8 int4 codes n0..n7 of one 32-bit word as the fp16 pairs (1024 + n_j,
@@ -324,6 +363,13 @@ struct NeuronLayout {
 // neurons of CTA c: i = c + m G, m < own_count; tile k holds m in [32k, 32k + 32)
 PI_DEV int own_count(int f, int c, int G) { return c < f ? (f - 1 - c) / G + 1 : 0; }
 
+// k16 steps [ks0, ks1) of the rank taken by consumer warp w
+PI_DEV void warp_ks(int r, int w, int &ks0, int &ks1) {
+  const int ks = r / 16;
+  ks0 = w * ks / kConsumerWarps;
+  ks1 = (w + 1) * ks / kConsumerWarps;
+}
+
 // ---------------------------------------------------------------- producer
 // The whole producer warp runs this loop in lockstep with identical state;
 // lane 0 writes the slot descriptors and arms the mbarriers, and the bulk
@@ -339,8 +385,12 @@ PI_DEV void producer(Smem &S, const Args &a, int c, int G, int lane) {
   const NeuronLayout<WT, ACT> NL(d);
   const int GN = min(kMaxGN, kSlotBytes / (int)NL.bytes);
   const unsigned rb = wrow_bytes<WT>(d), sb = srow_bytes<WT>(d);
+  const unsigned p2b = (unsigned)r * 2u;
+  const int M = a.p2_main;                       // rows of every CTA in the tensor map
+  const int left_tile = (c < f - M * G) ? M / kTN : -1;  // tile holding this CTA's leftover row m = M
   constexpr int CPN = (ACT == ACT_SWIGLU ? 3 : 2) * (WT == W_INT4 ? 2 : 1);  // copies per neuron
   const bool want_mask = a.idx != nullptr || a.count != nullptr;
+  const unsigned long long lim = a.wait_ns;
   unsigned pn = 0;   // items issued
   int k = 0;         // own tiles issued
   int hk = 0;        // own tiles harvested
@@ -352,7 +402,6 @@ PI_DEV void producer(Smem &S, const Args &a, int c, int G, int lane) {
   auto harvest = [&]() {
     const int s = S.tile_item[hk] % kSlots;
     const unsigned bits = S.tbits[s];
-    const int fired = __popc(bits);
     if (lane == 0) {
       unsigned b = bits;
       int t = act_tail;
@@ -373,7 +422,6 @@ PI_DEV void producer(Smem &S, const Args &a, int c, int G, int lane) {
       b &= b - 1u;
       added += (c + (hk * kTN + q) * G >= a.H) ? 1 : 0;
     }
-    (void)fired;
     act_tail += added;
     ++hk;
     __syncwarp();
@@ -387,7 +435,7 @@ PI_DEV void producer(Smem &S, const Args &a, int c, int G, int lane) {
   auto acquire = [&](int &s) -> bool {
     s = (int)(pn % kSlots);
     const unsigned par = ((pn / kSlots) & 1u) ^ 1u;
-    if (!mbar_wait(&S.empty[s], par, a.status)) {
+    if (!mbar_wait(&S.empty[s], par, a.status, lim)) {
       if (lane == 0) S.abort_flag = 1;
       return false;
     }
@@ -442,7 +490,7 @@ PI_DEV void producer(Smem &S, const Args &a, int c, int G, int lane) {
     return true;
   };
 
-  // 1. this CTA's rows of P1
+  // 1. this CTA's rows of P1, then an L2 prefetch of all its P2 rows
   for (int j = j0; ok && j < j1; j += rpi) {
     const int n = min(rpi, j1 - j);
     int s;
@@ -457,30 +505,28 @@ PI_DEV void producer(Smem &S, const Args &a, int c, int G, int lane) {
     }
     ++pn;
   }
-  // 2. predictor tiles and gather rows
+  // 2. predictor tiles, then gather rows.  Tiles go first: they decide which
+  // rows are needed, so the last tile's fired neurons are not left for the
+  // end of the stream
   while (ok) {
     while (hk < k && tile_done(hk)) harvest();
-    if (taken < act_tail) {
-      const int n = min(GN, act_tail - taken);
-      ok = issue_gather(&S.act[taken], n);
-      taken += n;
-      continue;
-    }
     if (k < nown) {
       const int rows = min(kTN, nn - k * kTN);
       int s;
       if (!(ok = acquire(s))) break;
-      const unsigned rbp = (unsigned)r * 2u;
       if (lane == 0) {
         S.meta[s].type = IT_P2;
         S.meta[s].n = rows;
         S.meta[s].first = k;
-        S.tbits[s] = 0u;
         S.tile_item[k] = (int)pn;
-        mbar_arrive_tx(&S.full[s], (unsigned)rows * rbp);
+        const bool main = k * kTN < M, left = k == left_tile;
+        mbar_arrive_tx(&S.full[s], (main ? (unsigned)kTN * p2b : 0u) + (left ? p2b : 0u));
+        // one tensor copy for the tile's rows c + m G, m in [32k, min(32k + 32, M))
+        if (main) tma_load_4d(S.ring[s], &a.tm_p2, 0, k * kTN, 0, c, &S.full[s]);
+        // the leftover row c + M G (when c < f - M G), plain, after the box
+        if (left) bulk_g2s(S.ring[s] + (size_t)kTN * p2b, a.p2 + (size_t)(c + M * G) * r, p2b, &S.full[s]);
       }
       __syncwarp();
-      if (lane < rows) bulk_g2s(S.ring[s] + lane * rbp, a.p2 + (size_t)(c + (k * kTN + lane) * G) * r, rbp, &S.full[s]);
       ++pn;
       // dense hot prefix: the tile's prefix neurons (the smallest ids), now
       int ms[kMaxGN], ng = 0;
@@ -496,10 +542,16 @@ PI_DEV void producer(Smem &S, const Args &a, int c, int G, int lane) {
       ++k;
       continue;
     }
+    if (taken < act_tail) {
+      const int n = min(GN, act_tail - taken);
+      ok = issue_gather(&S.act[taken], n);
+      taken += n;
+      continue;
+    }
     if (hk == nown) break;  // every tile harvested and every fired id issued
     // wait for the consumers to finish the oldest unharvested tile
     const unsigned it = (unsigned)S.tile_item[hk];
-    if (!mbar_wait(&S.empty[it % kSlots], (it / kSlots) & 1u, a.status)) {
+    if (!mbar_wait(&S.empty[it % kSlots], (it / kSlots) & 1u, a.status, lim)) {
       if (lane == 0) S.abort_flag = 1;
       ok = false;
       break;
@@ -507,7 +559,7 @@ PI_DEV void producer(Smem &S, const Args &a, int c, int G, int lane) {
     harvest();
   }
   // 3. end of stream (also after an abort, so consumers stop)
-  __threadfence();  // mask words visible before the consumers' grid barrier
+  __threadfence();  // mask words visible before the consumers publish partials
   int s;
   if (acquire(s)) {
     if (lane == 0) {
@@ -523,7 +575,7 @@ PI_DEV void producer(Smem &S, const Args &a, int c, int G, int lane) {
 // ---------------------------------------------------------------- kernel
 // CPT: column chunks per consumer thread (d <= CPT * 256 * EC)
 template <int WT, int ACT, int CPT>
-__global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Args a) {
+__global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_constant__ Args a) {
   // indexed directly (no integer round trip) so that every access stays in
   // the shared state space; bulk copies need only 16-byte alignment
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -534,11 +586,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Args a) {
   const int d = a.d, f = a.f, r = a.r;
   const int nwords = (f + 31) / 32;
   const int nn = own_count(f, c, G);
+  const unsigned long long lim = a.wait_ns;
 
   if (tid == 0) {
     for (int s = 0; s < kSlots; ++s) {
       mbar_init(&S.full[s], 1);
       mbar_init(&S.empty[s], kConsumerWarps);
+      S.tdone[s] = 0;
     }
     S.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -549,12 +603,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Args a) {
   // Programmatic dependent launch: the next step's grid may be scheduled
   // now, and its CTAs take SMs as this grid's CTAs leave.  The producer
   // streams weights only (P1 rows, P2 tiles, weight rows), which no earlier
-  // kernel writes, so it starts at once; the consumers wait for the
-  // preceding grid before reading the input or touching the workspace.
+  // kernel writes, so it starts at once; the consumers load this CTA's
+  // biases (weights too), then wait for the preceding grid before reading
+  // the input or touching the workspace.
   pdl_launch_dependents();
   if (warp == kConsumerWarps) {
     producer<WT, ACT>(S, a, c, G, lane);
     return;
+  }
+  constexpr int kBiasPer = kActCap / kConsumers;
+  float pbv[kBiasPer], bupv[kBiasPer];
+#pragma unroll
+  for (int q = 0; q < kBiasPer; ++q) {
+    const int m = tid + q * kConsumers;
+    pbv[q] = bupv[q] = 0.f;
+    if (m < nn) {
+      pbv[q] = __ldg(a.p_bias + c + (size_t)m * G);
+      if (ACT == ACT_RELU) bupv[q] = __ldg(a.b_up + c + (size_t)m * G);
+    }
   }
   pdl_wait();
 
@@ -572,7 +638,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Args a) {
   int coff[CPT];  // clamped chunk index
 #pragma unroll
   for (int q = 0; q < CPT; ++q) coff[q] = min(tid + q * kConsumers, nch - 1);
+  unsigned tag = 0;
   if (a.stack) {
+    tag = ld_relaxed_u32(a.epoch) + 1u;
     const float *x = reinterpret_cast<const float *>(a.in);
     double ss = 0.0;
     for (int k = tid; k < d; k += kConsumers) {
@@ -613,6 +681,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Args a) {
         uh[q][j] = valid ? v : make_uint4(0u, 0u, 0u, 0u);
       }
     }
+    tag = ld_relaxed_u32(a.epoch) + 1u;  // in flight together with the loads of u
   }
   // int4 dots take u in the (k, k+4) pair order of q8_pairs_biased, and the
   // chunk sums of u for the 1032 (= 1024 + 8) bias of the unpacked codes
@@ -641,23 +710,28 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Args a) {
 #pragma unroll
     for (int e = 0; e < EC; ++e) y[q][e] = 0.f;
 
-  // biases of this CTA's own neurons c + m G, one round trip
-  for (int m = tid; m < nn; m += kConsumers) {
-    const int i = c + m * G;
-    S.own_pbias[m / kTN][m % kTN] = __ldg(a.p_bias + i);
-    if (ACT == ACT_RELU) S.own_bup[m / kTN][m % kTN] = __ldg(a.b_up + i);
+#pragma unroll
+  for (int q = 0; q < kBiasPer; ++q) {
+    const int m = tid + q * kConsumers;
+    if (m < nn) {
+      S.own_pbias[m / kTN][m % kTN] = pbv[q];
+      S.own_bup[m / kTN][m % kTN] = bupv[q];
+    }
   }
-  // clear the fired-bit words (CTA c clears words c, c + G, ...); the first
-  // grid barrier orders this before any CTA sets bits
-  if (a.idx != nullptr || a.count != nullptr)
+  // clear the fired-bit words (CTA c clears words c, c + G, ...); a grid
+  // barrier orders this before any CTA sets bits
+  if (a.idx != nullptr || a.count != nullptr) {
     for (int w = c + tid * G; w < nwords; w += kConsumers * G) a.mask32[w] = 0u;
+    consumer_sync();
+    if (tid == 0 && !grid_barrier(a.bar, G, c, a.status, lim)) S.abort_flag = 1;
+  }
 
   unsigned n = 0;   // items consumed
   unsigned nr = 0;  // reductions done (parity of the red buffer)
   bool alive = true;
   auto wait_full = [&](int &s) -> bool {
     s = (int)(n % kSlots);
-    if (!mbar_wait(&S.full[s], (n / kSlots) & 1u, a.status)) {
+    if (!mbar_wait(&S.full[s], (n / kSlots) & 1u, a.status, lim)) {
       S.abort_flag = 1;
       return false;
     }
@@ -669,7 +743,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Args a) {
     ++n;
   };
 
-  // ---- P1 items: this CTA's slice of h (rows past the item alias row 0)
+  // ---- P1 items: this CTA's slice of h (rows past the item alias row 0),
+  // published as tagged words
   for (int it = 0; it < n_p1 && alive; ++it) {
     int s;
     if (!(alive = wait_full(s))) break;
@@ -697,33 +772,87 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Args a) {
     release(s);
     consumer_sync();
     ++nr;
-    if (tid < rows) {
+    if (tid < rows && c != a.withhold) {
       float t = 0.f;
 #pragma unroll
       for (int w = 0; w < kConsumerWarps; ++w) t += S.red[par][w][tid];
-      a.h[jf + tid] = t;
+      st_tagged(a.hx + jf + tid, tagged(t, tag));
     }
   }
-  // ---- h is complete once every CTA got here
-  consumer_sync();
-  if (tid == 0) {
-    if (!grid_barrier(a.bar, G, c, a.status)) S.abort_flag = 1;
+  // ---- h of every CTA: each warp gathers the slice of the rank its tensor-
+  // core steps use (lane: 4 consecutive entries), polling the tags
+  int ks0, ks1;
+  warp_ks(r, warp, ks0, ks1);
+  if (alive) {
+    // lane: entries e .. e + 3 (the warp's range is a multiple of 16 long).
+    // Two rounds of loads stay in flight: a new round goes out before the
+    // older one is checked, so a word published just after a round passed
+    // the L2 is seen half a round trip later.
+    const int e = ks0 * 16 + lane * 4;
+    bool done = e >= ks1 * 16;
+    unsigned long long wa[4], wb[4];
+    if (!done) {
+      ld_tagged2(a.hx + e, wa[0], wa[1]);
+      ld_tagged2(a.hx + e + 2, wa[2], wa[3]);
+    }
+    // issue a round into wn, then check the older round wo
+    auto round = [&](unsigned long long (&wo)[4], unsigned long long (&wn)[4]) {
+      if (done) return;
+      ld_tagged2(a.hx + e, wn[0], wn[1]);
+      ld_tagged2(a.hx + e + 2, wn[2], wn[3]);
+      if (tag_is(wo[0], tag) && tag_is(wo[1], tag) && tag_is(wo[2], tag) && tag_is(wo[3], tag)) {
+        S.h_s[e] = tagged_value(wo[0]);
+        S.h_s[e + 1] = tagged_value(wo[1]);
+        S.h_s[e + 2] = tagged_value(wo[2]);
+        S.h_s[e + 3] = tagged_value(wo[3]);
+        done = true;
+      }
+    };
+    // lane 0's clock decides for the warp, so the warp leaves together
+    const unsigned long long t0 = globaltimer();
+    auto expired = [&]() -> bool { return __shfl_sync(0xffffffffu, globaltimer() - t0 > lim ? 1 : 0, 0) != 0; };
+    for (;;) {
+      round(wa, wb);
+      if (__all_sync(0xffffffffu, done)) break;
+      round(wb, wa);
+      if (__all_sync(0xffffffffu, done)) break;
+      if (expired()) {
+        set_status(a.status, kStatusTimeout);
+        S.abort_flag = 1;
+        alive = false;
+        break;
+      }
+    }
+    __syncwarp();
   }
+  // a warp that gave up makes the whole CTA skip the stream, so that every
+  // consumer warp meets the same block barriers
   consumer_sync();
-  const int pch = r / 8;
-  for (int e = tid; e < r / 4; e += kConsumers)
-    reinterpret_cast<float4 *>(S.h_s)[e] = __ldcg(reinterpret_cast<const float4 *>(a.h) + e);
-  consumer_sync();
-  // predictor columns of this lane: chunks lane + 32 kk (8 fp16 each)
-  float hreg[4][8];
-  int hoff[4];
+  alive = alive && !S.abort_flag;
+  // B fragments of this warp's k16 steps: lanes 0-3 hold h_hi, lanes 4-7
+  // h_lo (columns 0 and 1 of B); every other lane holds zeros
+  uint32_t hb[kMaxKs][2];
 #pragma unroll
-  for (int kk = 0; kk < 4; ++kk) {
-    const int ch = lane + 32 * kk;
-    hoff[kk] = min(ch, pch - 1);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) hreg[kk][e] = (ch < pch) ? S.h_s[ch * 8 + e] : 0.f;
+  for (int i = 0; i < kMaxKs; ++i) {
+    hb[i][0] = hb[i][1] = 0u;
+    if (lane < 8 && ks0 + i < ks1 && alive) {
+      const int k0 = (ks0 + i) * 16 + 2 * (lane & 3), lo = lane >> 2;
+      hb[i][0] = h_part_pair(S.h_s[k0], S.h_s[k0 + 1], lo);
+      hb[i][1] = h_part_pair(S.h_s[k0 + 8], S.h_s[k0 + 9], lo);
+    }
   }
+  const int nks = ks1 - ks0;
+  // ldmatrix row addresses in the K-interleaved tile ([k / 8][row][k % 8],
+  // 16 bytes per row and chunk): lane L reads row L % 16 at k chunk
+  // 2 ks + L / 16; one k16 step is 2 chunks of 32 rows (1 KB), a 16-row half
+  // 256 bytes.  The CTA's leftover row (c < f - M G) sits, plain, after the
+  // box of its tile; the two lanes that read its position read it there.
+  const uint32_t a_off = ((uint32_t)(2 * ks0 + (lane >> 4)) * (uint32_t)kTN + (uint32_t)(lane & 15)) * 16u;
+  const int M = a.p2_main;
+  const int left_tile = (c < f - M * G) ? M / kTN : -1;
+  const int left_pos = M % kTN;
+  const bool left_lane = (lane & 15) == (left_pos & 15);
+  const uint32_t left_off = (uint32_t)kTN * 2u * (uint32_t)r + (uint32_t)(2 * ks0 + (lane >> 4)) * 16u;
 
   // ---- main stream
   while (alive) {
@@ -735,36 +864,56 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Args a) {
       break;
     }
     if (type == IT_P2) {
-      // rows warp + 8 q of the tile: all of this warp's loads first, then the
-      // dots, then one butterfly over the row sums
+      // this warp's k16 steps of both 16-row halves of the tile
       const int kl = S.meta[s].first, rows = S.meta[s].n;
-      constexpr int RPW = kTN / kConsumerWarps;
-      unsigned b = 0u;
-      uint4 wv[RPW][4];
+      float acc[2][4];
 #pragma unroll
-      for (int q = 0; q < RPW; ++q) {
-        const int row_i = warp + q * kConsumerWarps;
-        const __half *row = reinterpret_cast<const __half *>(S.ring[s]) + (size_t)min(row_i, rows - 1) * r;
+      for (int mb = 0; mb < 2; ++mb)
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) wv[q][kk] = *reinterpret_cast<const uint4 *>(row + hoff[kk] * 8);
+        for (int e = 0; e < 4; ++e) acc[mb][e] = 0.f;
+      const uint32_t slot = smem_u32(S.ring[s]);
+      const bool lt = kl == left_tile && left_lane;
+#pragma unroll
+      for (int i = 0; i < kMaxKs; ++i) {
+        if (i < nks) {
+#pragma unroll
+          for (int mb = 0; mb < 2; ++mb) {
+            uint32_t af[4];
+            const uint32_t ad = (lt && mb == (left_pos >> 4)) ? slot + left_off + (uint32_t)i * 32u
+                                                              : slot + a_off + (uint32_t)mb * 256u + (uint32_t)i * 1024u;
+            ldmatrix_x4(ad, af);
+            mma_16816(acc[mb], af, hb[i][0], hb[i][1]);
+          }
+        }
       }
-      float sv[RPW];
-#pragma unroll
-      for (int q = 0; q < RPW; ++q) {
-        float acc[4];
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) acc[kk] = dot8_h2(wv[q][kk], hreg[kk]);
-        sv[q] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+      // lanes 4g hold rows g and g + 8 of each half: s = D[.,0] + D[.,1]
+      if ((lane & 3) == 0) {
+        const int g = lane >> 2;
+        S.spart[s][warp][g] = acc[0][0] + acc[0][1];
+        S.spart[s][warp][g + 8] = acc[0][2] + acc[0][3];
+        S.spart[s][warp][g + 16] = acc[1][0] + acc[1][1];
+        S.spart[s][warp][g + 24] = acc[1][2] + acc[1][3];
       }
-      warp_sum_n<RPW>(sv);
-#pragma unroll
-      for (int q = 0; q < RPW; ++q) {
-        const int row_i = warp + q * kConsumerWarps;
-        if (row_i < rows && sv[q] + S.own_pbias[kl][row_i] > 0.f) b |= 1u << row_i;
+      __syncwarp();
+      int last = 0;
+      if (lane == 0) {
+        __threadfence_block();
+        last = atomicAdd(&S.tdone[s], 1) == kConsumerWarps - 1;
+        if (last) __threadfence_block();
       }
-      if (lane == 0 && b) {
-        atomicOr(&S.tbits[s], b);
-        atomicOr(&S.own_bits[kl], b);
+      last = __shfl_sync(0xffffffffu, last, 0);
+      if (last) {
+        // partial sums in warp order, then the bias: fire iff s > 0
+        float v = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) v += S.spart[s][w][lane];
+        const bool fire = lane < rows && v + S.own_pbias[kl][lane] > 0.f;
+        const unsigned b = __ballot_sync(0xffffffffu, fire);
+        if (lane == 0) {
+          S.tbits[s] = b;
+          S.own_bits[kl] = b;
+          S.tdone[s] = 0;
+        }
       }
       release(s);
       continue;
@@ -828,14 +977,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Args a) {
     // so the fired bits of the neurons' tiles are complete
     consumer_sync();
     ++nr;
-    // sum the 8 warps' partials: lane (g, w) = (lane / 8, lane % 8) loads
-    // warp w's partial of neuron g, a 3-step butterfly over the 8 lanes of a
-    // group adds them in a fixed order, and shuffles broadcast the sums
+    // sum the 16 warps' partials: lane (g, w) = (lane / 8, lane % 8) adds the
+    // partials of neuron g from warps w and w + 8, a 3-step butterfly over the
+    // 8 lanes of a group adds those in a fixed order, and shuffles broadcast
+    // the sums
     float a_l = 0.f;  // on lanes 8g: value of neuron g
     {
-      static_assert(kMaxGN * kConsumerWarps == 32, "one lane per (neuron, warp)");
-      float vu = S.red[par][lane & 7][2 * (lane >> 3)];
-      float vg = (ACT == ACT_SWIGLU) ? S.red[par][lane & 7][2 * (lane >> 3) + 1] : 0.f;
+      static_assert(kMaxGN * kConsumerWarps == 64, "one lane per neuron and warp pair");
+      float vu = S.red[par][lane & 7][2 * (lane >> 3)] + S.red[par][(lane & 7) + 8][2 * (lane >> 3)];
+      float vg = (ACT == ACT_SWIGLU)
+                     ? S.red[par][lane & 7][2 * (lane >> 3) + 1] + S.red[par][(lane & 7) + 8][2 * (lane >> 3) + 1]
+                     : 0.f;
 #pragma unroll
       for (int o = 1; o < 8; o <<= 1) {
         vu += __shfl_xor_sync(0xffffffffu, vu, o);
@@ -921,54 +1073,104 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Args a) {
     const unsigned long long t0 = globaltimer();
     while (globaltimer() - t0 < 1000000ull) __nanosleep(1000);
   }
-  // ---- partial of y
+  // ---- publish this CTA's partial of y as tagged words (after an abort too,
+  // so that the other CTAs' reductions complete)
+  if (a.idx != nullptr || a.count != nullptr) __threadfence();  // mask words before the partials
+  {
+    unsigned long long *pc = a.px + (size_t)c * d;
 #pragma unroll
-  for (int cq = 0; cq < CPT; ++cq) {
-    const int ch = tid + cq * kConsumers;
-    if (ch < nch) {
-      float4 *dst = reinterpret_cast<float4 *>(a.partial + (size_t)c * d + (size_t)ch * EC);
+    for (int cq = 0; cq < CPT; ++cq) {
+      const int ch = tid + cq * kConsumers;
+      if (ch < nch) {
 #pragma unroll
-      for (int e = 0; e < EC; e += 4) dst[e / 4] = make_float4(y[cq][e], y[cq][e + 1], y[cq][e + 2], y[cq][e + 3]);
-    }
-  }
-  consumer_sync();
-  if (tid == 0) {
-    if (!grid_barrier(a.bar, G, c, a.status)) S.abort_flag = 1;
-  }
-  consumer_sync();
-
-  // ---- column slice: sum of the G partials in CTA order
-  const int cw = (d + G - 1) / G;
-  const int c0 = min(d, c * cw), c1 = min(d, c0 + cw);
-  const int col_l = tid & 31, grp = tid >> 5;
-  for (int base = c0; base < c1; base += 32) {
-    const int col = base + col_l;
-    float sum = 0.f;
-    if (col < c1) {
-      constexpr int kMaxPer = 40;  // G <= 320
-      float v[kMaxPer];
-#pragma unroll
-      for (int q = 0; q < kMaxPer; ++q) {
-        const int cc = grp + q * kConsumerWarps;
-        v[q] = (cc < G) ? ld_cg(a.partial + (size_t)cc * d + col) : 0.f;
+        for (int e = 0; e < EC; e += 2)
+          st_tagged2(pc + (size_t)ch * EC + e, tagged(y[cq][e], tag), tagged(y[cq][e + 1], tag));
       }
-#pragma unroll
-      for (int q = 0; q < kMaxPer; ++q) sum += v[q];
     }
-    S.fin[grp][col_l] = sum;
-    consumer_sync();
-    if (grp == 0 && col < c1) {
-      float t = S.fin[0][col_l];
-#pragma unroll
-      for (int g = 1; g < kConsumerWarps; ++g) t += S.fin[g][col_l];
-      a.out[col] = (a.stack || a.accumulate) ? a.out[col] + t : t;
-    }
-    consumer_sync();
   }
 
-  // ---- ascending active ids (optional): CTA c writes the ids of words
-  // [c * tpc, (c + 1) * tpc) after the popcount of all earlier words
+  // ---- reduction.  The first R CTAs (R = ceil(d / kRedCols)) each sum a
+  // slice of kRedCols columns over all G partials; the others leave now, so
+  // the next launch's CTAs can take their SMs and start streaming weights
+  // while the reduction runs (the id lists, when asked for, need every CTA).
+  // Thread (grp, p) = (tid / 32, tid % 32) takes the column pair 2p of the
+  // slice from CTAs grp, grp + 8, ... (in that order), then the 8 group sums
+  // are added in group order: a fixed order, so y is deterministic.
+  const bool want_ids = a.idx != nullptr || a.count != nullptr;
+  const int n_red = (d + kRedCols - 1) / kRedCols;
+  if (c >= n_red && !want_ids) return;
+  if (c < n_red) {
+    constexpr int kGroups = kConsumers / (kRedCols / 2);
+    const int pr = tid % (kRedCols / 2), grp = tid / (kRedCols / 2);
+    const int col = c * kRedCols + 2 * pr;
+    float s0 = 0.f, s1 = 0.f;
+    bool timed_out = false;
+    if (col < d) {
+      // batches of kRedBatch partials: all loads of a batch go out before any
+      // tag is checked; the values wait in this thread's stage in the (now
+      // idle) ring until the batch is complete, then add in CTA order
+      float *stage = reinterpret_cast<float *>(S.ring[0]) + (size_t)tid * 2 * kRedBatch;
+      for (int qb = 0; grp + qb * kGroups < G; qb += kRedBatch) {
+        unsigned pending = 0u;
+#pragma unroll
+        for (int q = 0; q < kRedBatch; ++q)
+          if (grp + (qb + q) * kGroups < G) pending |= 1u << q;
+        const unsigned all = pending;
+        const unsigned long long t0 = globaltimer();
+        while (pending && !timed_out) {
+          unsigned long long w0[kRedBatch], w1[kRedBatch];
+#pragma unroll
+          for (int q = 0; q < kRedBatch; ++q)
+            if ((pending >> q) & 1u) ld_tagged2(a.px + (size_t)(grp + (qb + q) * kGroups) * d + col, w0[q], w1[q]);
+#pragma unroll
+          for (int q = 0; q < kRedBatch; ++q) {
+            if (((pending >> q) & 1u) && tag_is(w0[q], tag) && tag_is(w1[q], tag)) {
+              stage[2 * q] = tagged_value(w0[q]);
+              stage[2 * q + 1] = tagged_value(w1[q]);
+              pending &= ~(1u << q);
+            }
+          }
+          if (pending) {
+            if (globaltimer() - t0 > lim) {
+              set_status(a.status, kStatusTimeout);
+              timed_out = true;
+            } else {
+              __nanosleep(32);
+            }
+          }
+        }
+        for (int q = 0; q < kRedBatch; ++q) {
+          if (((all >> q) & 1u) && !((pending >> q) & 1u)) {
+            s0 += stage[2 * q];
+            s1 += stage[2 * q + 1];
+          }
+        }
+      }
+    }
+    S.fin[grp][2 * pr] = s0;
+    S.fin[grp][2 * pr + 1] = s1;
+    consumer_sync();
+    if (tid < kRedCols && c * kRedCols + tid < d) {
+      float t = S.fin[0][tid];
+#pragma unroll
+      for (int g = 1; g < kGroups; ++g) t += S.fin[g][tid];
+      const int oc = c * kRedCols + tid;
+      a.out[oc] = (a.stack || a.accumulate) ? a.out[oc] + t : t;
+    }
+  }
+  // every CTA has read the epoch (its partial carries this launch's tag):
+  // advance it for the next launch on this workspace
+  if (c == 0 && tid == 0) st_relaxed_u32(a.epoch, tag);
+
+  // ---- ascending active ids (optional): after a grid barrier, CTA c writes
+  // the ids of words [c * tpc, (c + 1) * tpc) after the popcount of all
+  // earlier words
   if (a.idx != nullptr || a.count != nullptr) {
+    consumer_sync();
+    if (tid == 0) {
+      if (!grid_barrier(a.bar, G, c, a.status, lim)) S.abort_flag = 1;
+    }
+    consumer_sync();
     const int tpc = (nwords + G - 1) / G;
     const int t0 = min(nwords, c * tpc), t1 = min(nwords, t0 + tpc);
     int before = 0, total = 0;

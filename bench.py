@@ -67,6 +67,11 @@ def parse(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-seconds", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-workers", type=int, default=64,
+                    help="oracle processes of the all-core CPU baseline (at most the host's cores; 0 skips it)")
+    ap.add_argument("--stack-config", default="opt30b_stack_f16",
+                    help="stacked workload timed as the line's 'stack' object at batch 1 ('none' skips it)")
+    ap.add_argument("--stack-steps", type=int, default=200)
     ap.add_argument("--json-out", default=None)
     ap.add_argument("--stack", action="store_true",
                     help="time pi_decode_ffn_stack through all layers of a stacked config (tokens/s)")
@@ -338,7 +343,10 @@ def bench_ours(args, world, rank, local):
             pair_bytes[(r, t)] = step_bytes(cfg, B, len(union))
     assert pb.pi_get_device_status(ws) == 0
 
-    # graphs: one of S = lcm(R, T) steps, plus single-step graphs for a remainder
+    # graphs: one of S = lcm(R, T) consecutive steps (the schedule's period),
+    # plus one graph of the first n steps for a remainder n, so that a run of
+    # K steps is K // S replays of the period and at most one more launch, and
+    # consecutive steps overlap through programmatic dependent launch
     S = int(np.lcm(R, T))
     sched = [(j % R, j % T) for j in range(S)]
 
@@ -350,23 +358,23 @@ def bench_ours(args, world, rank, local):
         for j in range(S):  # eager warm-up before capture
             step(j)
     stream.synchronize()
-    big = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(big, stream=stream):
-        for j in range(S):
-            step(j)
-    singles = []
-    for j in range(S):
+
+    def capture(n):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
-            step(j)
-        singles.append(g)
+            for j in range(n):
+                step(j)
+        return g
+
+    period = capture(S)
+    heads = {n: capture(n) for n in {args.warmup % S, args.steps % S} if n}
 
     def run(nsteps):
         with torch.cuda.stream(stream):
             for _ in range(nsteps // S):
-                big.replay()
-            for j in range(nsteps % S):
-                singles[j].replay()
+                period.replay()
+            if nsteps % S:
+                heads[nsteps % S].replay()
 
     run(args.warmup)
     torch.cuda.synchronize()
@@ -469,7 +477,11 @@ def bench_ours(args, world, rank, local):
                    "batch": B, "d_model": cfg.d, "d_ffn": cfg.f, "rank": cfg.r, "replicas": R, "tokens": T,
                    "l2": f"{R} rotating seeded replicas ({sum(l.nbytes() for l in layers) / 1e9:.1f} GB) > L2",
                    "bytes_per_step": nbytes / args.steps, "parallelism": f"replicas x{world}",
-                   "bias_norm": cfg.bias_norm, "hot_mode": args.hot_mode},
+                   "bias_norm": cfg.bias_norm, "hot_mode": args.hot_mode,
+                   "outputs": "y per step; the timed calls pass no idx/count, so the ascending global id list "
+                              "(step 2's optional output) is not written inside the timed region",
+                   "graphs": f"one CUDA graph per {S} consecutive steps (remainder: one graph of the first "
+                             f"steps), consecutive launches overlapping through programmatic dependent launch"},
         "roofline": {"bound": "hbm", "achieved": per_gpu, "peak": peak, "unit": "GB/s", "frac": per_gpu / peak,
                      "traffic": (profiled_traffic(f"decode_fused_kernel_{cfg.name}_batch{B}.md")
                                  if kernels_per_step(cfg, B) == 1 else None),
@@ -485,12 +497,57 @@ def bench_ours(args, world, rank, local):
         "gpu_launches": kernels_per_step(cfg, B) * args.steps,
         "clocks": clk.summary(),
     }
+    if args.stack_config != "none":
+        line["stack"] = stack_summary(args, world, rank, local)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n, csec, cbytes = oracle_run(layers[0].to("cpu"), cfg, toks_host, args.cpu_seconds, 10 ** 9)
+        host = layers[0].to("cpu")
+        del layers, handles
+        n, csec, cbytes = oracle_run(host, cfg, toks_host, args.cpu_seconds, 10 ** 9)
         line["cpu_baseline"] = {"value": cbytes / csec / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
                                 "sample": f"{n} whole tokens of replica 0, one host thread",
                                 "us_per_layer": csec / n * 1e6}
+        workers = min(args.cpu_workers, os.cpu_count() or 1)
+        if workers > 1:
+            line["cpu_baseline_all_cores"] = oracle_all_cores(host, cfg, toks_host, args.cpu_seconds, workers)
     return line
+
+
+def oracle_all_cores(host, cfg, toks_host, seconds, workers):
+    """The oracle as it stands, one spawned process per core, each on whole
+    tokens of the same layer (shared through memory-mapped files), for about
+    ``seconds``; aggregate GB/s = all processes' bytes over the wall time."""
+    import shutil
+    from oracle import timing
+    d = tempfile.mkdtemp(prefix="pi_oracle_")
+    try:
+        meta = timing.save_layer(host.host_arrays(), toks_host.numpy(), d)
+        res = timing.run_all_cores(d, meta, seconds, workers)
+    finally:
+        shutil.rmtree(d, ignore_errors=True)
+    B = toks_host.shape[1]
+    nbytes = sum(step_bytes(cfg, B, u) for u in res["unions"])
+    n = len(res["unions"])
+    return {"value": nbytes / res["wall"] / 1e9, "unit": "GB/s", "cores": res["workers"],
+            "host_cpu_count": os.cpu_count(), "kind": "oracle",
+            "sample": f"{n} whole tokens of replica 0 over {res['wall']:.1f} s, one single-threaded oracle "
+                      f"process per core ({res['workers']} processes)",
+            "us_per_layer_per_process": res["wall"] * res["workers"] / n * 1e6}
+
+
+def stack_summary(args, world, rank, local):
+    """Batch-1 FFN-stack decode of ``--stack-config`` (every layer, RMS norm,
+    predictor, sparse FFN, residual add), for the main line's 'stack' object."""
+    import copy
+    a = copy.copy(args)
+    a.config, a.batch, a.tokens = args.stack_config, 1, 4
+    a.steps, a.warmup = args.stack_steps, max(3, args.stack_steps // 10)
+    st = bench_stack(a, world, rank, local)
+    torch.cuda.empty_cache()
+    return {"workload": st["config"]["workload"], "tokens_per_s": st["value"], "us_per_layer": st["us_per_layer"],
+            "steps": st["steps"], "warmup": st["warmup"], "layers": st["config"]["layers"],
+            "bytes_per_token": st["config"]["bytes_per_step"], "roofline": st["roofline"],
+            "gpu_launches_per_token": st["gpu_launches_per_step"], "clocks": st["clocks"],
+            "generation_s": st["config"]["generation_s"]}
 
 
 def bench_stack(args, world, rank, local):
@@ -579,6 +636,7 @@ def bench_stack(args, world, rank, local):
                    "bias_norm": cfg.bias_norm, "hot_mode": args.hot_mode},
         "roofline": {"bound": "hbm", "achieved": gbs / world, "peak": peak, "unit": "GB/s",
                      "frac": gbs / world / peak, "peak_source": "measured" if "hbm_gbs" in peaks else "fallback"},
+        "gpu_launches_per_step": L * (kernels_per_step(cfg, B) + (0 if kernels_per_step(cfg, B) == 1 else 1)),
         "clocks": clk.summary(),
     }
 

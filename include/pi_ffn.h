@@ -164,7 +164,7 @@ pi_status pi_decode_ffn_stack(const pi_ffn_t *layers, int L, float *x, int B, in
 
 /* Size in bytes of the library's file-scope device scratch array, the only
  * device memory pi_decode_ffn_static uses besides its arguments. */
-#define PI_STATIC_SCRATCH_BYTES (4u * 1024u * 1024u)
+#define PI_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
 
 /* pi_decode_ffn at batch 1 without a caller workspace and without allocating.
  * The pages have no counterpart: this is an integration entry point only.
@@ -181,22 +181,40 @@ pi_status pi_decode_ffn_stack(const pi_ffn_t *layers, int L, float *x, int B, in
  * optional [f] / [1] int32 outputs as in pi_predict; flags: PI_FFN_*.
  * dev_status: optional device int (4-byte aligned); when non-NULL it receives,
  * in stream order, this call's device-side status (PI_OK, PI_ERR_TIMEOUT, ...).
+ * It is the only way to see a device-side error of this entry point: there is
+ * no caller workspace to read with pi_get_device_status, and the next call
+ * clears the scratch status word.
  *
  * Limits and behaviour:
  *  - The layer's batch-1 scratch (status words, h, mask words, union lists
- *    and one d-float partial row per SM) must fit PI_STATIC_SCRATCH_BYTES;
- *    otherwise the call returns PI_ERR_WORKSPACE and launches nothing.  On a
- *    148-SM B200 this admits d_model <= 6928 at d_ffn = 16384 and rank 1024
- *    (an OPT-7B- or LLaMA-13B-shaped layer, not OPT-30B or LLaMA-70B).
- *  - The first call on each device does the set-up (looks up the array's
- *    device address with the device current), so make it before any stream
- *    capture.  Each call clears the scratch status and barrier words on the
- *    stream before its kernels.
+ *    and, per SM, one fp32 and one tagged 8-byte partial row of d entries)
+ *    must fit PI_STATIC_SCRATCH_BYTES; otherwise the call returns
+ *    PI_ERR_WORKSPACE and launches nothing.  On a 148-SM B200 this admits
+ *    d_model <= 9360 at d_ffn = 28672 and rank 1024, i.e. every OPT-7B- to
+ *    LLaMA2-70B-shaped layer (d_model <= 8192).
+ *  - The first call on each device (and again after a device reset) does
+ *    the set-up: it looks up the array's device address with the device
+ *    current.  Make that first call before any stream capture.  Each call
+ *    clears the scratch status and barrier words on the stream before its
+ *    kernels; the fused kernel's exchange words are never cleared (their
+ *    tags advance with every launch).
  *  - There is one scratch array per device: calls that overlap on the GPU
  *    (other streams, other host threads) race on it and give wrong results.
  *    Serialise them, e.g. on one stream. */
 pi_status pi_decode_ffn_static(pi_ffn_t h, const void *u, float *y, int32_t *idx, int32_t *count, unsigned flags,
                                int *dev_status, pi_stream_t stream);
+
+/* Test support for the device-side failure reporting; not part of the decode
+ * path (the pages have no counterpart).  It makes the following batch-1 fused
+ * launches of this process exercise their bounded waits without any fault:
+ * CTA withhold_cta does not publish its slice of the predictor's h, so every
+ * other CTA's wait for h runs out after limit_us microseconds; each launch
+ * then records PI_ERR_TIMEOUT in the workspace status word and completes (its
+ * outputs are unspecified).  withhold_cta = -1 with limit_us = 0 restores
+ * normal operation; limit_us alone (withhold_cta = -1) only shortens the
+ * limit.  Returns PI_ERR_INVALID_ARG for withhold_cta < -1, or for a withheld
+ * CTA without a limit.  Not thread-safe; set it while no call is running. */
+pi_status pi_debug_wait_fault(int withhold_cta, unsigned limit_us);
 
 /* Synchronise the stream, read and clear the workspace status word.  *code is
  * PI_OK or the first device-side error recorded since the last read. */

@@ -135,3 +135,11 @@ def test_static_entry_and_status_calls_check_arguments_first(lib):
         assert lib.pi_get_device_status(vp(0x100), None, None) == pb.PI_ERR_INVALID_ARG
     finally:
         lib.pi_ffn_destroy(h)
+
+
+def test_wait_fault_hook_validation(lib):
+    """The failure-reporting test hook rejects a CTA index below -1 and a
+    withheld slice without a wait limit; (-1, 0) restores normal runs."""
+    assert lib.pi_debug_wait_fault(-2, 0) == pb.PI_ERR_INVALID_ARG
+    assert lib.pi_debug_wait_fault(0, 0) == pb.PI_ERR_INVALID_ARG
+    assert lib.pi_debug_wait_fault(-1, 0) == pb.PI_OK

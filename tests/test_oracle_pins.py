@@ -465,6 +465,56 @@ def test_stack_zero_down_projection_keeps_x():
     assert np.array_equal(st["x"], x)
 
 
+
+def test_stack_three_layers_fold_one_layer_stacks():
+    """Invariant of the recurrence x_(l+1) = x_l + y_l(S_l): a three-layer
+    stack equals three one-layer stacks applied in turn, each on its own
+    layer's weights and on the x the previous one returned, with the same
+    per-layer traces (ids, counts, y).  The one-layer stack is itself pinned
+    to rmsnorm -> predict -> masked FFN above."""
+    cfg = inputs.CONFIGS["opt30b_stack_f16"].scaled(d=64, f=256, r=16, n_layers=3)
+    Ls = [_layer(inputs.make_layer(cfg, l, 6)) for l in range(3)]
+    x = inputs.make_tokens(cfg, 0, 2, 6).numpy()
+    st = oracle.stack(Ls, x)
+    xl = x
+    for l in range(3):
+        one = oracle.stack([Ls[l]], xl)
+        assert np.array_equal(st["y"][l], one["y"][0]), f"layer {l}: y"
+        assert np.array_equal(st["count"][l], one["count"][0]), f"layer {l}: counts"
+        for b in range(2):
+            assert np.array_equal(st["idx"][l][b], one["idx"][0][b]), f"layer {l} token {b}: ids"
+        xl = one["x"]
+    assert np.array_equal(st["x"], xl)
+    # the layers differ, so a stack that reused one layer's weights would not fold
+    assert not np.array_equal(st["y"][1], oracle.stack([Ls[0]], oracle.stack([Ls[0]], x)["x"])["y"][0])
+
+
+def test_stack_two_layers_closed_form():
+    """Hand-derived two-layer stack (d = 8, two neurons per layer, identity
+    predictor so that s = W1 u + b exactly).  x0 = (8, 8, 0, ..., 0) has
+    mean square 16, so u0 = x0 / 4 = (2, 2, 0, ...) (the 1e-6 of the norm
+    vanishes in the float32 rounding of sqrt(16.000001)).  Layer 0: neuron 0
+    reads u_0 with bias -1 (pre-activation 1, fires), neuron 1 reads u_1 with
+    bias -3 (pre-activation -1, does not fire); W2T_0 = 8 (0, 0, 1, 1, 1, 1,
+    1, 1), so x1 = (8, ..., 8), whose mean square is 64: u1 = (1, ..., 1).
+    Layer 1: neuron 0 reads u_3 with bias 0.5 (fires, value 1.5) into
+    W2T_0 = 2 e_7; neuron 1 reads -u_4 with bias 0.5 (pre-activation -0.5).
+    So x2 = (8, 8, 8, 8, 8, 8, 8, 11).  Reusing layer 0's weights in layer 1
+    (pre-activation 1 - 1 = 0 does not fire) or feeding x0 instead of x1
+    (value 0.5) gives another x2."""
+    d = 8
+    e = np.eye(d, dtype=np.float32)
+    L0 = _manual_layer(np.stack([e[0], e[1]]), np.stack([8 * (1 - e[0] - e[1]), np.zeros(d, np.float32)]),
+                       np.array([-1.0, -3.0], np.float32), wtype="f16")
+    L1 = _manual_layer(np.stack([e[3], -e[4]]), np.stack([2 * e[7], np.ones(d, np.float32)]),
+                       np.array([0.5, 0.5], np.float32), wtype="f16")
+    x0 = np.array([[8, 8, 0, 0, 0, 0, 0, 0]], np.float32)
+    st = oracle.stack([L0, L1], x0)
+    assert np.array_equal(st["x"], np.array([[8, 8, 8, 8, 8, 8, 8, 11]], np.float32))
+    assert [list(st["idx"][l][0]) for l in range(2)] == [[0], [0]]
+    assert np.array_equal(st["y"][0][0], [0, 0, 8, 8, 8, 8, 8, 8])
+    assert np.array_equal(st["y"][1][0], [0, 0, 0, 0, 0, 0, 0, 3])
+
 # ---------------------------------------------------------------- generator checks
 
 @pytest.mark.parametrize("name,mean_p", [("opt7b_f16", 0.10), ("opt30b_stack_f16", 0.03),
