@@ -269,10 +269,11 @@ def pi_decode_ffn_stack(layers: Sequence[FfnLayer], x: torch.Tensor, ws: torch.T
                                      *_wsargs(ws), _stream(stream)), "pi_decode_ffn_stack")
 
 
-def pi_debug_wait_fault(withhold_cta: int = -1, limit_us: int = 0):
-    """Test support: batch-1 fused launches withhold one CTA's slice of h and
-    wait at most ``limit_us`` (see the header); (-1, 0) restores normal runs."""
-    _check(lib().pi_debug_wait_fault(int(withhold_cta), int(limit_us)), "pi_debug_wait_fault")
+def pi_debug_wait_fault(withhold_row: int = -1, limit_us: int = 0):
+    """Test support: batch-1 fused launches never publish entry ``withhold_row``
+    of h and wait at most ``limit_us`` (see the header); (-1, 0) restores
+    normal runs."""
+    _check(lib().pi_debug_wait_fault(int(withhold_row), int(limit_us)), "pi_debug_wait_fault")
 
 
 def pi_get_device_status(ws: torch.Tensor, stream=None) -> int:

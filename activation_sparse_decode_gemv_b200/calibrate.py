@@ -26,6 +26,16 @@ down rows, their int4 scales, the P2 rows and the biases) by one
 permutation; P1 is not per neuron and stays.  The FFN output is a sum over
 neurons, so it is unchanged up to the order of that sum, and a token's
 predicted set maps through the permutation.
+
+Predictor sizing (the summary page's Interesting ideas I3: each layer's
+predictor is sized by how predictable the layer is, within an accuracy
+target; its Key points quote a ~0.4% cosine shift of the layer outputs for
+the trained predictors): ``truncate_predictor`` keeps the leading r
+components of the factors, and ``size_rank`` picks the smallest candidate
+rank whose outputs stay within a mean cosine shift of a reference (the
+exact ReLU mask, or the full predictor) on calibration tokens.  The FFN
+evaluator and the predictors are callables again: the library's
+pi_predict / pi_sparse_ffn on the device, or the oracle in the tests.
 """
 from __future__ import annotations
 
@@ -144,3 +154,81 @@ def map_sets(sets: List[np.ndarray], perm: np.ndarray) -> List[np.ndarray]:
     inv = np.empty_like(np.asarray(perm, np.int64))
     inv[perm] = np.arange(len(perm))
     return [np.sort(inv[np.asarray(s, np.int64)]).astype(np.int32) for s in sets]
+
+
+# --------------------------------------------------------------------------
+# predictor sizing
+# --------------------------------------------------------------------------
+
+def truncate_predictor(lt: LayerTensors, rank: int) -> LayerTensors:
+    """The layer with a rank-``rank`` predictor: the leading ``rank`` rows of
+    P1 and columns of P2.  The generator's factors are P1 = V_r^T and
+    P2 = U_r Sigma_r of a truncated SVD in descending singular-value order, so
+    the cut is the rank-``rank`` truncated SVD of the same matrix.  The bias
+    and every FFN tensor stay."""
+    if rank < 1 or rank > lt.r:
+        raise ValueError(f"rank must be in [1, {lt.r}]")
+    cfg = dataclasses.replace(lt.cfg, r=int(rank))
+    return dataclasses.replace(lt, cfg=cfg, p1=lt.p1[:rank].contiguous(), p2=lt.p2[:, :rank].contiguous())
+
+
+def cosine_shift(y: np.ndarray, y_ref: np.ndarray) -> np.ndarray:
+    """1 - cos(y_b, y_ref_b) per token (0 where both are zero, 1 where only one is)."""
+    y, y_ref = np.atleast_2d(np.asarray(y, np.float64)), np.atleast_2d(np.asarray(y_ref, np.float64))
+    num = np.sum(y * y_ref, axis=1)
+    den = np.linalg.norm(y, axis=1) * np.linalg.norm(y_ref, axis=1)
+    both0 = (np.linalg.norm(y, axis=1) == 0) & (np.linalg.norm(y_ref, axis=1) == 0)
+    out = np.where(den > 0, 1.0 - num / np.where(den > 0, den, 1.0), 1.0)
+    return np.where(both0, 0.0, out)
+
+
+def set_recall(pred: Sequence[np.ndarray], ref: Sequence[np.ndarray]) -> float:
+    """Mean over tokens of |pred & ref| / |ref| (tokens with an empty ref count as 1)."""
+    vals = []
+    for p, r in zip(pred, ref):
+        r = np.asarray(r)
+        vals.append(1.0 if r.size == 0 else np.intersect1d(np.asarray(p), r).size / r.size)
+    return float(np.mean(vals)) if vals else 1.0
+
+
+@dataclasses.dataclass
+class RankChoice:
+    rank: int                 # chosen rank (the largest candidate when none meets the target)
+    met: bool                 # whether the chosen rank meets the target
+    table: List[dict]         # per candidate: rank, mean/max cosine shift, recall, mean set size
+
+
+def size_rank(ranks: Sequence[int], predict_at: Callable[[int, torch.Tensor], Sequence[np.ndarray]],
+              ffn: Callable[[torch.Tensor, Sequence[np.ndarray]], np.ndarray],
+              reference: Callable[[torch.Tensor], Sequence[np.ndarray]], batches: Iterable[torch.Tensor],
+              max_shift: float = 0.004) -> RankChoice:
+    """Smallest rank among ``ranks`` whose predicted sets keep the mean cosine
+    shift of the FFN output against the ``reference`` sets at or below
+    ``max_shift`` over the calibration ``batches``.
+
+    ``predict_at(r, u)`` returns the rank-r predictor's sets for tokens u,
+    ``ffn(u, sets)`` the layer output [B x d] over given sets, and
+    ``reference(u)`` the reference sets (the exact ReLU mask, or the full
+    predictor's)."""
+    batches = list(batches)
+    ranks = sorted(set(int(r) for r in ranks))
+    if not ranks or not batches:
+        raise ValueError("need candidate ranks and calibration tokens")
+    refs = [(u, reference(u)) for u in batches]
+    y_refs = [ffn(u, sets) for u, sets in refs]
+    table = []
+    choice = None
+    for r in ranks:
+        shifts, recalls, sizes = [], [], []
+        for (u, ref), y_ref in zip(refs, y_refs):
+            sets = predict_at(r, u)
+            shifts.append(cosine_shift(ffn(u, sets), y_ref))
+            recalls.append(set_recall(sets, ref))
+            sizes.append(np.mean([len(s) for s in sets]))
+        sh = np.concatenate(shifts)
+        row = dict(rank=r, mean_shift=float(sh.mean()), max_shift=float(sh.max()), recall=float(np.mean(recalls)),
+                   mean_set=float(np.mean(sizes)))
+        table.append(row)
+        if choice is None and row["mean_shift"] <= max_shift:
+            choice = r
+    return RankChoice(rank=choice if choice is not None else ranks[-1], met=choice is not None, table=table)

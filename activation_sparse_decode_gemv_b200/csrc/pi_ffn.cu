@@ -609,8 +609,8 @@ pi_status run_ffn_tc(const pi_ffn *h, const void *u, int B, float *out, int accu
 // ---------------------------------------------------------------- fused batch-1 path
 namespace F = pi::fused;
 
-// Test support (pi_debug_wait_fault): a CTA that withholds its slice of h and
-// a shorter limit for every bounded wait of the fused kernel.
+// Test support (pi_debug_wait_fault): an entry of h that is never published,
+// and a shorter limit for every bounded wait of the fused kernel.
 struct WaitFault {
   int withhold = -1;
   unsigned long long limit_ns = 0;  // 0: the kernel's default
@@ -978,10 +978,10 @@ pi_status pi_decode_ffn_static(pi_ffn_t h, const void *u, float *y, int32_t *idx
   return PI_OK;
 }
 
-pi_status pi_debug_wait_fault(int withhold_cta, unsigned limit_us) {
-  if (withhold_cta < -1) return PI_ERR_INVALID_ARG;
-  if (withhold_cta >= 0 && limit_us == 0) return PI_ERR_INVALID_ARG;
-  g_wait_fault.withhold = withhold_cta;
+pi_status pi_debug_wait_fault(int withhold_row, unsigned limit_us) {
+  if (withhold_row < -1) return PI_ERR_INVALID_ARG;
+  if (withhold_row >= 0 && limit_us == 0) return PI_ERR_INVALID_ARG;
+  g_wait_fault.withhold = withhold_row;
   g_wait_fault.limit_ns = (unsigned long long)limit_us * 1000ull;
   return PI_OK;
 }

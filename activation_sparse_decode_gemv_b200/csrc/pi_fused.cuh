@@ -133,7 +133,7 @@ struct Args {
   int32_t *idx;    // optional ascending active ids [f]
   int32_t *count;  // optional [1]
   unsigned long long wait_ns;  // limit of every bounded wait
-  int withhold;    // CTA that does not publish its slice of h (-1: none); exercises the bounded waits
+  int withhold;    // entry of h that is never published (-1: none); exercises the bounded waits
 };
 
 // ---------------------------------------------------------------- PTX helpers
@@ -772,7 +772,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
     release(s);
     consumer_sync();
     ++nr;
-    if (tid < rows && c != a.withhold) {
+    if (tid < rows && jf + tid != a.withhold) {
       float t = 0.f;
 #pragma unroll
       for (int w = 0; w < kConsumerWarps; ++w) t += S.red[par][w][tid];

@@ -77,6 +77,8 @@ def parse(argv=None):
                     help="time pi_decode_ffn_stack through all layers of a stacked config (tokens/s)")
     ap.add_argument("--hot-mode", default="auto", choices=sorted(HOT_MODE_FLAGS),
                     help="read the hot prefix densely, by index, or as the library decides (adds to --flags)")
+    ap.add_argument("--rank", type=int, default=0,
+                    help="cut every layer's predictor to its leading RANK components (0: the config's rank)")
     ap.add_argument("--bias-norm", default=None, choices=["pred", "w1"],
                     help="predictor bias scale of the generated layers (default: the config's)")
     args = ap.parse_args(argv)
@@ -92,6 +94,30 @@ def config_of(args) -> inputs.Config:
     """The workload of --config, with the --bias-norm override."""
     cfg = inputs.CONFIGS[args.config]
     return cfg.scaled(bias_norm=args.bias_norm) if args.bias_norm else cfg
+
+
+RAMP_SECONDS = 0.03
+
+
+def clock_ramp(work) -> float:
+    """Untimed replays of ``work`` for RAMP_SECONDS before the warm-up steps,
+    so that a short timed run starts at the clocks of a busy GPU (a timed
+    region of a few hundred microseconds right after the idle setup would
+    otherwise include the ramp).  Returns the seconds spent."""
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < RAMP_SECONDS:
+        work()
+        torch.cuda.synchronize()
+    return time.perf_counter() - t0
+
+
+def sized(args, lt):
+    """The layer with its predictor cut to ``--rank`` leading components
+    (the predictor sizing of the calibration module), or as generated."""
+    if not args.rank or args.rank == lt.r:
+        return lt
+    from activation_sparse_decode_gemv_b200 import calibrate
+    return calibrate.truncate_predictor(lt, args.rank)
 
 
 # ----------------------------------------------------------------------------- distributed plumbing
@@ -291,7 +317,8 @@ def bench_reference(args, world, rank):
     if rank != 0:
         return None
     cfg = config_of(args)
-    lt = inputs.make_layer(cfg, 0, seed=1000, device="cuda" if torch.cuda.is_available() else "cpu").to("cpu")
+    lt = sized(args, inputs.make_layer(cfg, 0, seed=1000, device="cuda" if torch.cuda.is_available() else "cpu")).to("cpu")
+    cfg = lt.cfg
     toks = torch.stack([inputs.layer_input(cfg, inputs.make_tokens(cfg, t, args.batch, seed=1000))
                         for t in range(args.tokens)])
     # warm-up: the requested count of whole tokens, at most 3 (one oracle token
@@ -320,7 +347,8 @@ def bench_ours(args, world, rank, local):
     cfg = config_of(args)
     B, R, T = args.batch, args.replicas, args.tokens
     seed = 1000 + rank
-    layers = [inputs.make_layer(cfg, r, seed=seed, device=dev) for r in range(R)]
+    layers = [sized(args, inputs.make_layer(cfg, r, seed=seed, device=dev)) for r in range(R)]
+    cfg = layers[0].cfg
     handles = [pb.FfnLayer.from_tensors(lt) for lt in layers]
     ws = pb.make_workspace(handles, B, dev)
     toks_host = torch.stack([inputs.layer_input(cfg, inputs.make_tokens(cfg, t, B, seed=seed)) for t in range(T)])
@@ -376,6 +404,12 @@ def bench_ours(args, world, rank, local):
             if nsteps % S:
                 heads[nsteps % S].replay()
 
+    # every graph the timed run launches has been launched once before: a
+    # graph's first launch uploads it to the device
+    with torch.cuda.stream(stream):
+        for g in heads.values():
+            g.replay()
+    ramp_s = clock_ramp(lambda: run(S))
     run(args.warmup)
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -481,10 +515,12 @@ def bench_ours(args, world, rank, local):
                    "outputs": "y per step; the timed calls pass no idx/count, so the ascending global id list "
                               "(step 2's optional output) is not written inside the timed region",
                    "graphs": f"one CUDA graph per {S} consecutive steps (remainder: one graph of the first "
-                             f"steps), consecutive launches overlapping through programmatic dependent launch"},
+                             f"steps), consecutive launches overlapping through programmatic dependent launch",
+                   "untimed_before_warmup": f"each graph launched once, then {ramp_s * 1e3:.0f} ms of replays "
+                                            f"of the {S}-step graph (clock ramp)"},
         "roofline": {"bound": "hbm", "achieved": per_gpu, "peak": peak, "unit": "GB/s", "frac": per_gpu / peak,
                      "traffic": (profiled_traffic(f"decode_fused_kernel_{cfg.name}_batch{B}.md")
-                                 if kernels_per_step(cfg, B) == 1 else None),
+                                 if kernels_per_step(cfg, B) == 1 and not args.rank else None),
                      "algorithmic_bytes_per_launch": nbytes / args.steps,
                      "kernel": ("decode_fused_kernel (the whole step is one launch)" if kernels_per_step(cfg, B) == 1
                                 else f"whole decode step ({kernels_per_step(cfg, B)} kernels)"),
@@ -563,7 +599,8 @@ def bench_stack(args, world, rank, local):
     B, L, T = args.batch, cfg.n_layers, args.tokens
     seed = 3000 + rank
     t0 = time.perf_counter()
-    layers = [inputs.make_layer(cfg, l, seed=seed, device=dev) for l in range(L)]
+    layers = [sized(args, inputs.make_layer(cfg, l, seed=seed, device=dev)) for l in range(L)]
+    cfg = layers[0].cfg
     gen_s = time.perf_counter() - t0
     handles = [pb.FfnLayer.from_tensors(lt) for lt in layers]
     ws = pb.make_workspace(handles, B, dev)
@@ -603,6 +640,10 @@ def bench_stack(args, world, rank, local):
             for j in range(n):
                 graphs[j % T].replay()
 
+    # every graph the timed run launches has been launched once before: a
+    # graph's first launch uploads it to the device
+    run(T)
+    clock_ramp(lambda: run(T))
     run(args.warmup)
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

@@ -207,14 +207,15 @@ pi_status pi_decode_ffn_static(pi_ffn_t h, const void *u, float *y, int32_t *idx
 /* Test support for the device-side failure reporting; not part of the decode
  * path (the pages have no counterpart).  It makes the following batch-1 fused
  * launches of this process exercise their bounded waits without any fault:
- * CTA withhold_cta does not publish its slice of the predictor's h, so every
- * other CTA's wait for h runs out after limit_us microseconds; each launch
- * then records PI_ERR_TIMEOUT in the workspace status word and completes (its
- * outputs are unspecified).  withhold_cta = -1 with limit_us = 0 restores
- * normal operation; limit_us alone (withhold_cta = -1) only shortens the
- * limit.  Returns PI_ERR_INVALID_ARG for withhold_cta < -1, or for a withheld
- * CTA without a limit.  Not thread-safe; set it while no call is running. */
-pi_status pi_debug_wait_fault(int withhold_cta, unsigned limit_us);
+ * entry withhold_row of the predictor's h (0 <= withhold_row < rank) is never
+ * published, so every CTA's wait for h runs out after limit_us microseconds;
+ * each launch then records PI_ERR_TIMEOUT in the workspace status word and
+ * completes (its outputs are unspecified).  withhold_row = -1 with
+ * limit_us = 0 restores normal operation; limit_us alone (withhold_row = -1)
+ * only shortens the limit.  Returns PI_ERR_INVALID_ARG for withhold_row < -1,
+ * or for a withheld entry without a limit.  Not thread-safe; set it while no
+ * call is running. */
+pi_status pi_debug_wait_fault(int withhold_row, unsigned limit_us);
 
 /* Synchronise the stream, read and clear the workspace status word.  *code is
  * PI_OK or the first device-side error recorded since the last read. */

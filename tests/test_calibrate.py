@@ -137,3 +137,62 @@ def test_firing_counts_validates_predictor_output():
         calibrate.firing_counts(lambda u: [np.array([16]), np.array([])], [u], 16)
     c, n = calibrate.firing_counts(lambda u: [np.array([0, 3]), np.array([3])], [u, u], 4)
     assert n == 4 and c.tolist() == [2, 0, 0, 4]
+
+
+# ---------------------------------------------------------------- predictor sizing
+
+def test_truncate_predictor_keeps_leading_components():
+    cfg = inputs.CONFIGS["opt7b_f16"].scaled(d=128, f=256, r=64)
+    lt = inputs.make_layer(cfg, 0, seed=5)
+    t = calibrate.truncate_predictor(lt, 16)
+    assert t.r == 16 and t.p1.shape == (16, 128) and t.p2.shape == (256, 16)
+    assert torch.equal(t.p1, lt.p1[:16]) and torch.equal(t.p2, lt.p2[:, :16])
+    assert torch.equal(t.p_bias, lt.p_bias) and torch.equal(t.w_up, lt.w_up)
+    assert torch.equal(calibrate.truncate_predictor(lt, 64).p2, lt.p2)
+    for bad in (0, 65):
+        with pytest.raises(ValueError):
+            calibrate.truncate_predictor(lt, bad)
+    # the factors are in descending singular-value order: the leading
+    # component of P2 carries the most energy
+    col = torch.linalg.vector_norm(lt.p2.double(), dim=0)
+    assert torch.all(col[:-1] >= col[1:] - 1e-3)
+
+
+def test_cosine_shift_and_recall_closed_forms():
+    y = np.array([[1.0, 0.0], [0.0, 0.0], [1.0, 1.0], [0.0, 0.0]])
+    r = np.array([[2.0, 0.0], [0.0, 0.0], [1.0, -1.0], [1.0, 0.0]])
+    assert np.allclose(calibrate.cosine_shift(y, r), [0.0, 0.0, 1.0, 1.0])
+    assert calibrate.set_recall([np.array([1, 2, 3])], [np.array([2, 3, 4, 5])]) == 0.5
+    assert calibrate.set_recall([np.array([], np.int32)], [np.array([], np.int32)]) == 1.0
+
+
+def test_size_rank_against_the_exact_relu_mask():
+    """On a small ReLU layer, the sizing compares each truncated predictor's
+    outputs with those over the exact mask (pre-activation > 0): the shift
+    falls as the rank grows, the full-rank predictor is within the pages'
+    0.4% shift, and the choice is the smallest rank that meets the target."""
+    cfg = inputs.CONFIGS["opt7b_f16"].scaled(d=128, f=512, r=128)
+    lt = inputs.make_layer(cfg, 0, seed=9)
+    L = _host(lt)
+    hosts = {r: _host(calibrate.truncate_predictor(lt, r)) for r in (8, 32, 128)}
+    batches = [_u(cfg, step, 32, 9) for step in range(2)]
+
+    def predict_at(r, u):
+        return oracle.predict(hosts[r], u.numpy())["idx"]
+
+    def ffn(u, sets):
+        return oracle.ffn_masked(L, u.numpy(), sets)
+
+    def exact(u):
+        pre = oracle.relu_preact(L, u.numpy())
+        return [np.nonzero(p > 0)[0].astype(np.int32) for p in pre]
+
+    ch = calibrate.size_rank([8, 32, 128], predict_at, ffn, exact, batches)
+    shifts = [row["mean_shift"] for row in ch.table]
+    assert shifts[0] > shifts[1] > shifts[2]
+    assert ch.table[2]["mean_shift"] <= 0.004 and ch.table[2]["recall"] > 0.95
+    assert ch.met and ch.rank == min(row["rank"] for row in ch.table if row["mean_shift"] <= 0.004)
+    loose = calibrate.size_rank([8, 32, 128], predict_at, ffn, exact, batches, max_shift=1.0)
+    assert loose.rank == 8 and loose.met
+    none = calibrate.size_rank([8, 32], predict_at, ffn, exact, batches, max_shift=-1.0)
+    assert none.rank == 32 and not none.met

@@ -52,3 +52,47 @@ def test_calibrate_with_pi_predict_then_decode_matches_oracle(cuda_device):
     for B_chk in (1, 4):
         u = inputs.layer_input(cfg, inputs.make_tokens(cfg, 100, B_chk, seed=71))
         check_layer(lr.to("cpu"), u, g)
+
+
+def test_size_rank_on_the_device(cuda_device):
+    """Predictor sizing with the library's own calls: each truncated predictor
+    through pi_predict, the FFN output over its sets through pi_sparse_ffn,
+    against the full rank-1024 predictor's sets on an OPT-7B-shaped layer.
+    The full rank reproduces the reference exactly (shift 0, recall 1), the
+    shift falls as the rank grows, and the choice is the smallest candidate
+    within the 0.4% cosine shift."""
+    dev = cuda_device
+    cfg = inputs.CONFIGS["opt7b_f16"]
+    lt = inputs.make_layer(cfg, 0, seed=73, device=dev)
+    ranks = (256, 512, 1024)
+    cut = {r: calibrate.truncate_predictor(lt, r) for r in ranks}
+    layers = {r: pb.FfnLayer.from_tensors(cut[r]) for r in ranks}
+    B = 8
+    ws = pb.make_workspace(list(layers.values()), B, dev)
+
+    def predict_at(r, u):
+        idx = torch.empty((u.shape[0], cfg.f), dtype=torch.int32, device=dev)
+        cnt = torch.empty((u.shape[0],), dtype=torch.int32, device=dev)
+        pb.pi_predict(layers[r], u, idx, cnt, ws)
+        idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+        return [idx[b, :cnt[b]] for b in range(len(cnt))]
+
+    def ffn(u, sets):
+        idx = torch.zeros((u.shape[0], cfg.f), dtype=torch.int32)
+        cnt = torch.zeros((u.shape[0],), dtype=torch.int32)
+        for b, s in enumerate(sets):
+            idx[b, :len(s)] = torch.from_numpy(np.asarray(s, np.int32))
+            cnt[b] = len(s)
+        y = torch.empty((u.shape[0], cfg.d), device=dev)
+        pb.pi_sparse_ffn(layers[1024], u, idx.to(dev), cnt.to(dev), y, ws)
+        return y.cpu().numpy()
+
+    batches = [inputs.layer_input(cfg, inputs.make_tokens(cfg, step, B, seed=79)).to(dev) for step in range(2)]
+    ch = calibrate.size_rank(ranks, predict_at, ffn, lambda u: predict_at(1024, u), batches)
+    assert pb.pi_get_device_status(ws) == 0
+    full = ch.table[-1]
+    assert full["rank"] == 1024 and full["mean_shift"] <= 1e-12 and full["recall"] == 1.0
+    shifts = [row["mean_shift"] for row in ch.table]
+    assert shifts[0] >= shifts[1] >= shifts[2]
+    assert ch.met and ch.rank == min(row["rank"] for row in ch.table if row["mean_shift"] <= 0.004)
+    print("rank sizing table:", ch.table)
