@@ -14,9 +14,10 @@
 //               A = the tile's rows, B = h split into h_hi = fp16(h) and
 //               h_lo = fp16(h - h_hi) as the first two of the 8 columns, so
 //               s = D[:,0] + D[:,1] carries h to about 22 bits.  Each warp
-//               takes one eighth of the rank; the last warp to finish a tile
-//               adds the eight partial sums in warp order and sets the fired
-//               bits, so no block barrier is needed per tile.
+//               takes one sixteenth of the rank and leaves its partial sums
+//               in shared memory; the producer, which waits for the slot
+//               anyway, adds them in warp order and sets the fired bits, so a
+//               tile costs the consumers neither a barrier nor an atomic.
 //   GATHER      up (+gate) and down rows of 1-4 neurons: dot with u,
 //               activation, then y += a * W2T_i in per-thread registers
 //   DONE        end of the stream
@@ -76,6 +77,7 @@ enum ItemType : int { IT_P1 = 0, IT_P2 = 1, IT_GATHER = 2, IT_DONE = 3 };
 
 struct SlotMeta {
   int type, n, first;
+  int tslot;  // gather item of dense hot-prefix rows: slot of their tile's partial scores; else -1
   int ids[kMaxGN];
 };
 
@@ -84,15 +86,12 @@ struct Smem {
   SlotMeta meta[kSlots];
   unsigned long long full[kSlots];
   unsigned long long empty[kSlots];
-  unsigned tbits[kSlots];              // fired bits of the tile in a slot
-  int tdone[kSlots];                   // consumer warps done with the tile in a slot
-  unsigned own_bits[kMaxOwnTiles];     // fired bits of this CTA's tiles
   int act[kActCap];                    // fired ids (index mode), producer-owned
   int tile_item[kMaxOwnTiles];         // item number each own tile was issued as
   float own_pbias[kMaxOwnTiles][kTN];  // predictor bias of this CTA's neurons
   float own_bup[kMaxOwnTiles][kTN];    // ReLU bias b1 of this CTA's neurons
   float h_s[kMaxR];                    // h, gathered from all CTAs
-  float spart[kSlots][kConsumerWarps][kTN];  // per-warp partial scores of a tile
+  float spart[kSlots][kConsumerWarps][kTN];  // per-warp partial scores of the tile in a slot
   float red[2][kConsumerWarps][2 * kMaxGN];
   double dred[kConsumerWarps];
   float fin[kConsumers / (kRedCols / 2)][kRedCols + 1];
@@ -398,10 +397,16 @@ PI_DEV void producer(Smem &S, const Args &a, int c, int G, int lane) {
   int taken = 0;     // fired own indices issued as gather items
   bool ok = true;
 
-  // fired bits of own tile hk are final once its slot's empty phase completed
+  // own tile hk's partial scores are complete once its slot's empty phase
+  // completed: lane q adds the 16 warps' partials of row q in warp order,
+  // then the bias; fire iff s > 0
   auto harvest = [&]() {
     const int s = S.tile_item[hk] % kSlots;
-    const unsigned bits = S.tbits[s];
+    const int rows = min(kTN, nn - hk * kTN);
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) v += S.spart[s][w][lane];
+    const unsigned bits = __ballot_sync(0xffffffffu, lane < rows && v + S.own_pbias[hk][lane] > 0.f);
     if (lane == 0) {
       unsigned b = bits;
       int t = act_tail;
@@ -442,8 +447,9 @@ PI_DEV void producer(Smem &S, const Args &a, int c, int G, int lane) {
     while (hk < k && (unsigned)S.tile_item[hk] + kSlots <= pn) harvest();
     return true;
   };
-  // gather item: own indices ms[0..n); lane j issues copy j
-  auto issue_gather = [&](const int *ms, int n) -> bool {
+  // gather item: own indices ms[0..n); lane j issues copy j.  tslot: slot of
+  // the tile of dense hot-prefix rows (their bits are not known yet), else -1
+  auto issue_gather = [&](const int *ms, int n, int tslot) -> bool {
     int s;
     if (!acquire(s)) return false;
     if (lane == 0) {
@@ -451,6 +457,7 @@ PI_DEV void producer(Smem &S, const Args &a, int c, int G, int lane) {
       m.type = IT_GATHER;
       m.n = n;
       m.first = 0;
+      m.tslot = tslot;
       for (int g = 0; g < n; ++g) m.ids[g] = ms[g];
       mbar_arrive_tx(&S.full[s], NL.bytes * (unsigned)n);
     }
@@ -529,22 +536,23 @@ PI_DEV void producer(Smem &S, const Args &a, int c, int G, int lane) {
       __syncwarp();
       ++pn;
       // dense hot prefix: the tile's prefix neurons (the smallest ids), now
+      const int ts = (int)((pn - 1) % kSlots);
       int ms[kMaxGN], ng = 0;
       for (int q = 0; ok && q < rows; ++q) {
         if (c + (k * kTN + q) * G >= a.H) break;
         ms[ng++] = k * kTN + q;
         if (ng == GN) {
-          ok = issue_gather(ms, ng);
+          ok = issue_gather(ms, ng, ts);
           ng = 0;
         }
       }
-      if (ok && ng) ok = issue_gather(ms, ng);
+      if (ok && ng) ok = issue_gather(ms, ng, ts);
       ++k;
       continue;
     }
     if (taken < act_tail) {
       const int n = min(GN, act_tail - taken);
-      ok = issue_gather(&S.act[taken], n);
+      ok = issue_gather(&S.act[taken], n, -1);
       taken += n;
       continue;
     }
@@ -592,12 +600,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
     for (int s = 0; s < kSlots; ++s) {
       mbar_init(&S.full[s], 1);
       mbar_init(&S.empty[s], kConsumerWarps);
-      S.tdone[s] = 0;
     }
     S.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  for (int k = tid; k < kMaxOwnTiles; k += blockDim.x) S.own_bits[k] = 0u;
   __syncthreads();
 
   // Programmatic dependent launch: the next step's grid may be scheduled
@@ -865,7 +871,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
     }
     if (type == IT_P2) {
       // this warp's k16 steps of both 16-row halves of the tile
-      const int kl = S.meta[s].first, rows = S.meta[s].n;
+      const int kl = S.meta[s].first;
       float acc[2][4];
 #pragma unroll
       for (int mb = 0; mb < 2; ++mb)
@@ -894,32 +900,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
         S.spart[s][warp][g + 16] = acc[1][0] + acc[1][1];
         S.spart[s][warp][g + 24] = acc[1][2] + acc[1][3];
       }
-      __syncwarp();
-      int last = 0;
-      if (lane == 0) {
-        __threadfence_block();
-        last = atomicAdd(&S.tdone[s], 1) == kConsumerWarps - 1;
-        if (last) __threadfence_block();
-      }
-      last = __shfl_sync(0xffffffffu, last, 0);
-      if (last) {
-        // partial sums in warp order, then the bias: fire iff s > 0
-        float v = 0.f;
-#pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) v += S.spart[s][w][lane];
-        const bool fire = lane < rows && v + S.own_pbias[kl][lane] > 0.f;
-        const unsigned b = __ballot_sync(0xffffffffu, fire);
-        if (lane == 0) {
-          S.tbits[s] = b;
-          S.own_bits[kl] = b;
-          S.tdone[s] = 0;
-        }
-      }
       release(s);
       continue;
     }
-    // IT_GATHER: neurons past the item alias neuron 0 and get a zero value
+    // IT_GATHER: neurons past the item alias neuron 0 and get a zero value.
+    // Index-mode items hold fired neurons only; for dense hot-prefix rows the
+    // lanes 8g work out membership from their tile's partial scores (same
+    // sum, same order as the producer's), before the barrier below, since the
+    // next tile in that slot may overwrite them once every warp has passed it
     const int ng = S.meta[s].n;
+    bool member = true;
+    {
+      const int ts = S.meta[s].tslot;
+      const int g_l = lane >> 3;
+      if (ts >= 0 && (lane & 7) == 0 && g_l < ng) {
+        const int m = S.meta[s].ids[g_l];
+        float v = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) v += S.spart[ts][w][m % kTN];
+        member = v + S.own_pbias[m / kTN][m % kTN] > 0.f;
+      }
+    }
     const uint8_t *nd[kMaxGN];
 #pragma unroll
     for (int g = 0; g < kMaxGN; ++g) nd[g] = S.ring[s] + (g < ng ? g : 0) * NL.bytes;
@@ -998,7 +999,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
       if ((lane & 7) == 0 && g_l < ng) {
         const int m = S.meta[s].ids[g_l];  // own index: neuron c + m G
         const int kl = m / kTN;
-        if ((S.own_bits[kl] >> (m % kTN)) & 1u) {
+        if (member) {
           if (ACT == ACT_RELU)
             a_l = fmaxf(vu + S.own_bup[kl][m % kTN], 0.f);
           else
