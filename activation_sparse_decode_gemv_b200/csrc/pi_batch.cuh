@@ -1,0 +1,476 @@
+// pi_batch.cuh -- the FFN of a token batch of 2..8 over the union of the
+// tokens' predicted sets, as one persistent kernel per layer (PowerInfer
+// summary page: Summary, neuron-aware sparse operators; Interesting ideas I4,
+// kernels that read only the rows of the active neurons).
+//
+// Grid: one CTA per SM (all co-resident; the one grid-wide wait is bounded).
+// The union list (hot prefix first in dense mode) is the K of step 3 and the
+// reduction axis of step 4.  Both steps are small matrix products with the
+// batch as N = 8 columns, so they run on the tensor cores (mma.sync
+// m16n8k16, fp16 inputs, fp32 accumulation); the work is bound by HBM, and the
+// tensor cores only keep the instruction count per weight byte low.
+//
+// Step 3 (up / gate + activation).  CTA c takes the list positions
+// [chunk_begin(c), chunk_begin(c + 1)), in groups of 16 neurons (the MMA's M).
+// A unit is 64 elements of the 16 rows of a group.  The weight rows go from
+// HBM straight into registers: lane (g, q) of a warp loads 16 bytes at
+// elements 8q and 32 + 8q of rows g and g + 8, which is an A fragment once the
+// K order inside the unit is permuted the same way for the token operand (a
+// dot product does not depend on the order of its terms).  The tokens sit in
+// shared memory.  The CTA's units are split into 16 contiguous spans, one per
+// warp (stream-K inside the CTA); each warp leaves one partial per group it
+// touched in shared memory and the CTA adds them in warp order.  The
+// activation a (zero for tokens that did not predict the neuron) is stored as
+// two fp16 parts, a_hi = fp16(a) and a_lo = fp16(a - a_hi), so step 4 carries
+// a to about 22 bits.
+//
+// Step 4 (down).  y^T [d x 8] = W2T^T [d x list] * a [list x 8].  A unit is a
+// tile of 64 columns of y times 16 list positions; units are ordered tile by
+// tile and split into G contiguous spans (stream-K over CTAs), so every CTA
+// does the same amount of work and reads 128-byte row segments.  Inside a CTA
+// the warps take the units of a tile in turn and each keeps its own ring of 4
+// shared-memory stages filled with cp.async (16-byte copies, XOR-swizzled so
+// that ldmatrix.trans reads them without bank conflicts); the activations of
+// the unit's positions ride in the same stage.  A tile covered by one CTA is
+// written to y directly; a tile split between CTAs is finished by the last
+// CTA to arrive (per-tile counter), which adds the pieces in CTA order, so the
+// result does not depend on timing.  Counters reset themselves.
+#pragma once
+
+#include <cuda.h>
+
+#include "pi_device.cuh"
+#include "pi_fused.cuh"
+
+namespace pi {
+namespace batch {
+
+using fused::globaltimer;
+using fused::grid_barrier;
+using fused::mma_16816;
+using fused::smem_u32;
+
+constexpr int kWarps = 16;
+constexpr int kThreads = kWarps * 32;
+constexpr int kTok = 8;          // token columns (batches of 2..8; rows past B are zero)
+constexpr int kKStep = 64;       // elements of one step-3 unit
+constexpr int kTileCols = 64;    // columns of y per step-4 tile
+constexpr int kPosStep = 16;     // list positions per step-4 unit
+constexpr int kStages = 4;       // step-4 stages per warp
+constexpr int kRowBytes = kTileCols * 2;
+constexpr int kStageBytes = kPosStep * kRowBytes + 2 * kTok * kPosStep * 2;  // rows + a_hi + a_lo
+constexpr int kMaxLoc = 512;     // list positions one CTA takes in step 3
+constexpr int kMaxSlots = 3;     // groups one warp's step-3 span touches (kMaxLoc / 16 <= 32 groups)
+constexpr int kMaxTiles = 192;   // step-4 tiles (d <= 12288)
+constexpr int kPieceFloats = kTileCols * kTok;
+constexpr unsigned long long kWaitNs = 2000000000ull;
+
+struct Args {
+  const void *w_up, *w_gate, *w_down_t;
+  const float *b_up;
+  const __half *u;  // [B x d] fp16
+  int d, f, B;
+  const uint32_t *mask;  // [B x nwords] per-token mask words
+  int nwords;
+  const int32_t *ulist, *ucount, *uprefix;
+  int hot_dense, H;
+  __half *a_hi, *a_lo;  // [kTok x a_stride] activations by list position
+  int a_stride;
+  float *part;     // [G x 2 x kPieceFloats] pieces of split tiles
+  unsigned *ctr;   // [d / kTileCols] arrival counters, zero between launches
+  unsigned *bar;   // grid-barrier word
+  float *out;      // [B x d]
+  int accumulate;  // out += y instead of out = y
+  int *status;
+  unsigned long long wait_ns;
+};
+
+// dynamic shared memory: step 3 (tokens + warp partials) and step 4 (stages +
+// tile partials) use the same bytes, one after the other
+inline __host__ __device__ size_t step3_bytes(int d, int nmat) {
+  return (size_t)kTok * (2 * (size_t)d + 64) + (size_t)kWarps * kMaxSlots * nmat * 128 * 4;
+}
+inline __host__ __device__ size_t step4_bytes() {
+  return (size_t)kWarps * kStages * kStageBytes + (size_t)kWarps * kPieceFloats * 4;
+}
+inline __host__ __device__ size_t smem_bytes(int d, int nmat) {
+  const size_t a = step3_bytes(d, nmat), b = step4_bytes();
+  return a > b ? a : b;
+}
+
+// ---------------------------------------------------------------- PTX helpers
+PI_DEV void ldmatrix_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+PI_DEV void cp_async16(uint32_t dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+PI_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+PI_DEV void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+PI_DEV void st_shared_zero16(uint32_t dst) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
+}
+
+// number of list positions of the grid's list and the range of CTA c (the
+// same formulas as the CUDA-core gather kernel)
+PI_DEV int list_len(const int32_t *ucount, const int32_t *uprefix, int hot_dense, int H) {
+  const int U = *ucount;
+  return hot_dense ? H + (U - uprefix[H >> 5]) : U;
+}
+PI_DEV int list_begin(int c, int V, int G) { return (int)(((long long)c * V) / G); }
+
+// step-4 span of CTA c: units [span_lo(c), span_lo(c + 1)) of W
+PI_DEV long long span_lo(long long W, int c, int G) { return W * c / G; }
+// the CTA whose span holds unit x (the largest c with span_lo(c) <= x)
+PI_DEV int span_owner(long long W, long long x, int G) { return (int)(((x + 1) * G + W - 1) / W) - 1; }
+
+template <int ACT>
+__global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_constant__ Args a) {
+  constexpr int NM = ACT == ACT_SWIGLU ? 2 : 1;
+  constexpr int PD = ACT == ACT_SWIGLU ? 2 : 3;  // step-3 units in flight per warp
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ int ids_s[kMaxLoc];
+  __shared__ uint32_t memb_s[kMaxLoc];
+  __shared__ float bias_s[kMaxLoc];
+  __shared__ int last_s;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, q = lane & 3;
+  const int G = gridDim.x, c = blockIdx.x;
+  const int d = a.d, B = a.B;
+  const size_t rb = (size_t)d * 2;
+
+  pdl_wait();
+  const int V = list_len(a.ucount, a.uprefix, a.hot_dense, a.H);
+  const int upre_h = a.hot_dense ? a.uprefix[a.H >> 5] : 0;
+  auto vid = [&](int p) -> int { return a.hot_dense ? (p < a.H ? p : a.ulist[upre_h + (p - a.H)]) : a.ulist[p]; };
+
+  // ================================================================ step 3
+  const int pb = list_begin(c, V, G), pe = list_begin(c + 1, V, G);
+  const int nloc = pe - pb;
+  const int upitch = d + 32;  // halves; rows 64 bytes apart modulo 128
+  __half *u_s = reinterpret_cast<__half *>(smem);
+  float *red = reinterpret_cast<float *>(smem + (size_t)kTok * upitch * 2);
+  {
+    const int dch = d / 8;
+    for (int k = tid; k < kTok * dch; k += kThreads) {
+      const int t = k / dch, e = k - t * dch;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (t < B) v = *reinterpret_cast<const uint4 *>(a.u + (size_t)t * d + (size_t)e * 8);
+      *reinterpret_cast<uint4 *>(u_s + (size_t)t * upitch + (size_t)e * 8) = v;
+    }
+    for (int k = tid; k < nloc; k += kThreads) {
+      const int i = vid(pb + k);
+      uint32_t m = 0u;
+      for (int t = 0; t < B; ++t) m |= ((a.mask[(size_t)t * a.nwords + (i >> 5)] >> (i & 31)) & 1u) << t;
+      ids_s[k] = i;
+      memb_s[k] = m;
+      if (ACT == ACT_RELU) bias_s[k] = a.b_up[i];
+    }
+  }
+  __syncthreads();
+
+  const int ns = d / kKStep;
+  const int ng = (nloc + 15) >> 4;
+  const int T = ng * ns;
+  const int w0 = (int)((long long)T * warp / kWarps), w1 = (int)((long long)T * (warp + 1) / kWarps);
+  const int ja = w0 / ns;
+  {
+    struct Buf {
+      uint4 w[NM][4];  // [matrix][row g lo, row g hi, row g+8 lo, row g+8 hi]
+    };
+    auto load = [&](Buf &bf, int ui) {
+      const int j = ui / ns, s = ui - j * ns;
+      const int r0 = 16 * j + g, r1 = r0 + 8;
+      const size_t off = (size_t)s * (kKStep * 2) + (size_t)q * 16;
+#pragma unroll
+      for (int m = 0; m < NM; ++m) {
+        const char *W = reinterpret_cast<const char *>(m == 0 ? a.w_up : a.w_gate);
+        if (r0 < nloc) {
+          const char *p = W + (size_t)ids_s[r0] * rb + off;
+          bf.w[m][0] = ld_stream16(p);
+          bf.w[m][1] = ld_stream16(p + 64);
+        } else {
+          bf.w[m][0] = bf.w[m][1] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        if (r1 < nloc) {
+          const char *p = W + (size_t)ids_s[r1] * rb + off;
+          bf.w[m][2] = ld_stream16(p);
+          bf.w[m][3] = ld_stream16(p + 64);
+        } else {
+          bf.w[m][2] = bf.w[m][3] = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+    };
+    float acc[NM][4];
+#pragma unroll
+    for (int m = 0; m < NM; ++m)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[m][e] = 0.f;
+    auto compute = [&](const Buf &bf, int ui) {
+      const int j = ui / ns, s = ui - j * ns;
+      const __half *ur = u_s + (size_t)g * upitch + (size_t)s * kKStep + q * 8;
+      const uint4 ub0 = *reinterpret_cast<const uint4 *>(ur), ub1 = *reinterpret_cast<const uint4 *>(ur + 32);
+#pragma unroll
+      for (int m = 0; m < NM; ++m) {
+        const uint4 &x0 = bf.w[m][0], &x1 = bf.w[m][1], &y0 = bf.w[m][2], &y1 = bf.w[m][3];
+        {
+          const uint32_t A[4] = {x0.x, y0.x, x0.y, y0.y};
+          mma_16816(acc[m], A, ub0.x, ub0.y);
+        }
+        {
+          const uint32_t A[4] = {x0.z, y0.z, x0.w, y0.w};
+          mma_16816(acc[m], A, ub0.z, ub0.w);
+        }
+        {
+          const uint32_t A[4] = {x1.x, y1.x, x1.y, y1.y};
+          mma_16816(acc[m], A, ub1.x, ub1.y);
+        }
+        {
+          const uint32_t A[4] = {x1.z, y1.z, x1.w, y1.w};
+          mma_16816(acc[m], A, ub1.z, ub1.w);
+        }
+      }
+      if (s == ns - 1 || ui == w1 - 1) {  // end of this warp's part of group j
+#pragma unroll
+        for (int m = 0; m < NM; ++m) {
+          float *dst = red + ((size_t)((warp * kMaxSlots + (j - ja)) * NM + m) * 128) + lane * 4;
+          *reinterpret_cast<float4 *>(dst) = make_float4(acc[m][0], acc[m][1], acc[m][2], acc[m][3]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[m][e] = 0.f;
+        }
+      }
+    };
+    Buf buf[PD];
+#pragma unroll
+    for (int k = 0; k < PD - 1; ++k)
+      if (w0 + k < w1) load(buf[k], w0 + k);
+    for (int ui = w0; ui < w1; ui += PD) {
+#pragma unroll
+      for (int k = 0; k < PD; ++k) {
+        const int uk = ui + k;
+        if (uk < w1) {
+          if (uk + PD - 1 < w1) load(buf[(k + PD - 1) % PD], uk + PD - 1);
+          compute(buf[k], uk);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  // sums over the warps in warp order, activation, membership; a by position
+  for (int it = tid; it < ng * 128; it += kThreads) {
+    const int j = it >> 7, rm = (it >> 3) & 15, t = it & 7;
+    const int p = 16 * j + rm;
+    if (p >= nloc) continue;
+    const int ln = (rm & 7) * 4 + (t >> 1), e = (t & 1) + ((rm >> 3) << 1);
+    float x[NM];
+#pragma unroll
+    for (int m = 0; m < NM; ++m) x[m] = 0.f;
+    for (int w = 0; w < kWarps; ++w) {
+      const int lo = (int)((long long)T * w / kWarps), hi = (int)((long long)T * (w + 1) / kWarps);
+      if (lo >= hi) continue;
+      const int jlo = lo / ns, jhi = (hi - 1) / ns;
+      if (j < jlo || j > jhi) continue;
+#pragma unroll
+      for (int m = 0; m < NM; ++m) x[m] += red[(size_t)((w * kMaxSlots + (j - jlo)) * NM + m) * 128 + ln * 4 + e];
+    }
+    float av = 0.f;
+    if ((memb_s[p] >> t) & 1u) {
+      if constexpr (ACT == ACT_RELU)
+        av = fmaxf(x[0] + bias_s[p], 0.f);
+      else
+        av = silu(x[1]) * x[0];
+    }
+    const __half hi = __float2half_rn(av);
+    const __half lo = __float2half_rn(av - __half2float(hi));
+    a.a_hi[(size_t)t * a.a_stride + pb + p] = hi;
+    a.a_lo[(size_t)t * a.a_stride + pb + p] = lo;
+  }
+  // the positions past the list up to the next multiple of 16 read as zero
+  if (c == G - 1 && tid < kTok * kPosStep) {
+    const int t = tid / kPosStep, p = V + tid % kPosStep;
+    if (p < ((V + kPosStep - 1) / kPosStep) * kPosStep) {
+      a.a_hi[(size_t)t * a.a_stride + p] = __float2half_rn(0.f);
+      a.a_lo[(size_t)t * a.a_stride + p] = __float2half_rn(0.f);
+    }
+  }
+  __syncthreads();
+
+  // ================================================================ step 4
+  const int ntiles = d / kTileCols;
+  const int S = (V + kPosStep - 1) / kPosStep;
+  const long long W = (long long)ntiles * S;
+  const long long u0 = span_lo(W, c, G), u1 = span_lo(W, c + 1, G);
+  const uint32_t ring = smem_u32(smem) + (uint32_t)(warp * kStages * kStageBytes);
+  float *tred = reinterpret_cast<float *>(smem + (size_t)kWarps * kStages * kStageBytes);
+  const char *Wd = reinterpret_cast<const char *>(a.w_down_t);
+  const int ta = u0 < u1 ? (int)(u0 / S) : 0, tb = u0 < u1 ? (int)((u1 - 1) / S) : -1;
+  // units of tile t in this CTA's span: steps [sa, sb)
+  auto tile_steps = [&](int t, int &sa, int &sb) {
+    const long long lo = (long long)t * S, hi = lo + S;
+    sa = (int)((u0 > lo ? u0 : lo) - lo);
+    sb = (int)((u1 < hi ? u1 : hi) - lo);
+  };
+  auto warp_count = [&](int t) {
+    int sa, sb;
+    tile_steps(t, sa, sb);
+    return sb - sa > warp ? (sb - sa - warp + kWarps - 1) / kWarps : 0;
+  };
+  int K = 0;
+  for (int t = ta; t <= tb; ++t) K += warp_count(t);
+  // k-th unit of this warp -> (tile, step)
+  auto unit_of = [&](int k, int &t, int &s) {
+    for (t = ta; t <= tb; ++t) {
+      const int n = warp_count(t);
+      if (k < n) {
+        int sa, sb;
+        tile_steps(t, sa, sb);
+        s = sa + warp + k * kWarps;
+        return;
+      }
+      k -= n;
+    }
+  };
+  auto issue_acts = [&](int k) {
+    int t, s;
+    unit_of(k, t, s);
+    const uint32_t st = ring + (uint32_t)((k % kStages) * kStageBytes);
+    const int hl = lane >> 4, t8 = (lane >> 1) & 7, half = lane & 1;
+    const __half *src = (hl ? a.a_lo : a.a_hi) + (size_t)t8 * a.a_stride + (size_t)s * kPosStep + half * 8;
+    cp_async16(st + (uint32_t)(kPosStep * kRowBytes + hl * (kTok * kPosStep * 2) + t8 * 32 + half * 16), src);
+  };
+  auto issue = [&](int k, bool rows, bool acts) {
+    if (k < K) {
+      int t, s;
+      unit_of(k, t, s);
+      const uint32_t st = ring + (uint32_t)((k % kStages) * kStageBytes);
+      if (rows) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int row = (lane >> 3) + 4 * i, ch = lane & 7;
+          const int p = s * kPosStep + row;
+          const uint32_t dst = st + (uint32_t)(row * kRowBytes + ((ch ^ (row & 7)) << 4));
+          if (p < V)
+            cp_async16(dst, Wd + (size_t)vid(p) * rb + (size_t)t * kRowBytes + ch * 16);
+          else
+            st_shared_zero16(dst);
+        }
+      }
+      if (acts) issue_acts(k);
+    }
+    cp_async_commit();
+  };
+
+  // the first stages' weight rows do not depend on step 3: in flight during
+  // the grid-wide wait
+#pragma unroll
+  for (int k = 0; k < kStages - 1; ++k) issue(k, true, false);
+  if (tid == 0) grid_barrier(a.bar, G, c, a.status, a.wait_ns);
+  __syncthreads();
+  pdl_launch_dependents();
+  // their activations, as one more group
+  for (int k = 0; k < kStages - 1; ++k)
+    if (k < K) issue_acts(k);
+  cp_async_commit();
+
+  if (W == 0) {  // empty list: y = 0
+    if (!a.accumulate)
+      for (int k = c * kThreads + tid; k < B * d; k += G * kThreads) a.out[k] = 0.f;
+    return;
+  }
+
+  float acc_h[4][4], acc_l[4][4];
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc_h[mt][e] = acc_l[mt][e] = 0.f;
+  int k = 0;
+  for (int t = ta; t <= tb; ++t) {
+    const int nt = warp_count(t);
+    for (int n = 0; n < nt; ++n, ++k) {
+      if (k == 0)
+        cp_async_wait<0>();
+      else if (k == 1)
+        cp_async_wait<1>();
+      else
+        cp_async_wait<kStages - 2>();
+      __syncwarp();
+      const uint32_t st = ring + (uint32_t)((k % kStages) * kStageBytes);
+      const uint32_t ab = st + kPosStep * kRowBytes;
+      uint32_t bh0, bh1, bl0, bl1;
+      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(bh0) : "r"(ab + g * 32 + q * 4));
+      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(bh1) : "r"(ab + g * 32 + 16 + q * 4));
+      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(bl0) : "r"(ab + kTok * kPosStep * 2 + g * 32 + q * 4));
+      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(bl1) : "r"(ab + kTok * kPosStep * 2 + g * 32 + 16 + q * 4));
+      const int mi = lane >> 3, r = lane & 7, row = r + 8 * (mi >> 1);
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt) {
+        const int ch = 2 * mt + (mi & 1);
+        uint32_t A[4];
+        ldmatrix_x4_trans(st + (uint32_t)(row * kRowBytes + ((ch ^ r) << 4)), A);
+        mma_16816(acc_h[mt], A, bh0, bh1);
+        mma_16816(acc_l[mt], A, bl0, bl1);
+      }
+      __syncwarp();
+      issue(k + kStages - 1, true, true);
+    }
+    // this warp's partial of tile t
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt) {
+      float *dst = tred + (size_t)warp * kPieceFloats;
+      const int col = 16 * mt + g;
+      *reinterpret_cast<float2 *>(dst + col * kTok + 2 * q) =
+          make_float2(acc_h[mt][0] + acc_l[mt][0], acc_h[mt][1] + acc_l[mt][1]);
+      *reinterpret_cast<float2 *>(dst + (col + 8) * kTok + 2 * q) =
+          make_float2(acc_h[mt][2] + acc_l[mt][2], acc_h[mt][3] + acc_l[mt][3]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc_h[mt][e] = acc_l[mt][e] = 0.f;
+    }
+    __syncthreads();
+    // tile sum over the warps (in warp order); item = column * 8 + token
+    const int col = tid >> 3, tok = tid & 7;
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) v += tred[(size_t)w * kPieceFloats + tid];
+    const long long tlo = (long long)t * S, thi = tlo + S;
+    const int cf = span_owner(W, tlo, G), cl = span_owner(W, thi - 1, G);
+    float *y = a.out + (size_t)tok * d + (size_t)t * kTileCols + col;
+    if (cf == cl) {
+      if (tok < B) *y = a.accumulate ? *y + v : v;
+    } else {
+      const int slot = (t == ta) ? 0 : 1;
+      a.part[((size_t)c * 2 + slot) * kPieceFloats + tid] = v;
+      __threadfence();
+      __syncthreads();
+      if (tid == 0) {
+        int pieces = 0;
+        for (int cc = cf; cc <= cl; ++cc) pieces += span_lo(W, cc + 1, G) > span_lo(W, cc, G) ? 1 : 0;
+        const unsigned old = atomicAdd(&a.ctr[t], 1u);
+        last_s = (old == (unsigned)(pieces - 1)) ? 1 : 0;
+        if (last_s) {
+          a.ctr[t] = 0u;
+          __threadfence();
+        }
+      }
+      __syncthreads();
+      if (last_s) {
+        float s = 0.f;
+        for (int cc = cf; cc <= cl; ++cc) {
+          const long long clo = span_lo(W, cc, G), chi = span_lo(W, cc + 1, G);
+          if (chi <= clo) continue;
+          const int sl = (t == (int)(clo / S)) ? 0 : 1;
+          s += __ldcg(a.part + ((size_t)cc * 2 + sl) * kPieceFloats + tid);
+        }
+        if (tok < B) *y = a.accumulate ? *y + s : s;
+      }
+    }
+    __syncthreads();
+  }
+  cp_async_wait<0>();
+}
+
+}  // namespace batch
+}  // namespace pi

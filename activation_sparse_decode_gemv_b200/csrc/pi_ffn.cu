@@ -10,6 +10,7 @@
 #include <mutex>
 #include <new>
 
+#include "pi_batch.cuh"
 #include "pi_ffn.h"
 #include "pi_fused.cuh"
 #include "pi_kernels.cuh"
@@ -39,13 +40,18 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // Workspace layout for a call at batch B on layers with the given maxima.
 // [0, 256): status region: int status, int union count, grid-barrier word,
 // and (at byte 64) the epoch of the fused kernel's tagged words.
+// [256, 1024): the batch kernel's per-tile arrival counters (zero between
+// calls; the kernel restores them), at a place that does not move with B.
 // fx_h / fx_part: the fused kernel's tagged exchange words (h, partials of y);
 // no other kernel writes them, so a stale word can never carry a current tag.
 struct WsLayout {
-  size_t h, u, mask, uwords, uprefix, ulist, partial, fx_h, fx_part, total;
-  int G;
+  size_t h, u, mask, uwords, uprefix, ulist, partial, fx_h, fx_part, b_ahi, b_alo, b_part, total;
+  int G, a_stride;
 };
 constexpr size_t kEpochOffset = 64;
+constexpr size_t kBatchCtrOffset = 256;
+constexpr size_t kHeaderBytes = 1024;
+static_assert(kBatchCtrOffset + pi::batch::kMaxTiles * 4 <= kHeaderBytes, "batch counters fit the header");
 
 int device_sm_count() {
   int dev = 0, n = 0;
@@ -56,7 +62,7 @@ int device_sm_count() {
 
 WsLayout ws_layout(int dmax, int fmax, int rmax, int B, int G) {
   WsLayout L{};
-  size_t o = 256;
+  size_t o = kHeaderBytes;
   const size_t nw = (size_t)(fmax + 31) / 32;
   L.h = o;
   o = align_up(o + (size_t)B * rmax * 4, 256);
@@ -76,6 +82,18 @@ WsLayout ws_layout(int dmax, int fmax, int rmax, int B, int G) {
   o = align_up(o + (size_t)rmax * 8, 256);
   L.fx_part = o;
   o = align_up(o + (size_t)G * dmax * 8, 256);
+  // batch kernel: activations by list position (hi and lo parts) and the
+  // pieces of tiles split between CTAs
+  // (batches of 2 or more only)
+  L.a_stride = (int)align_up((size_t)fmax + pi::batch::kPosStep, 16);
+  L.b_ahi = L.b_alo = L.b_part = o;
+  if (B >= 2) {
+    o = align_up(o + (size_t)pi::batch::kTok * L.a_stride * 2, 256);
+    L.b_alo = o;
+    o = align_up(o + (size_t)pi::batch::kTok * L.a_stride * 2, 256);
+    L.b_part = o;
+    o = align_up(o + (size_t)G * 2 * pi::batch::kPieceFloats * 4, 256);
+  }
   L.total = o;
   L.G = G;
   return L;
@@ -224,6 +242,10 @@ struct Ws {
   unsigned *epoch() const { return reinterpret_cast<unsigned *>(base + kEpochOffset); }
   unsigned long long *fx_h() const { return reinterpret_cast<unsigned long long *>(base + L.fx_h); }
   unsigned long long *fx_part() const { return reinterpret_cast<unsigned long long *>(base + L.fx_part); }
+  __half *b_ahi() const { return reinterpret_cast<__half *>(base + L.b_ahi); }
+  __half *b_alo() const { return reinterpret_cast<__half *>(base + L.b_alo); }
+  float *b_part() const { return reinterpret_cast<float *>(base + L.b_part); }
+  unsigned *b_ctr() const { return reinterpret_cast<unsigned *>(base + kBatchCtrOffset); }
   unsigned char *uimg() const { return reinterpret_cast<unsigned char *>(tc + T.uimg); }
   unsigned char *uimg_perm() const { return reinterpret_cast<unsigned char *>(tc + T.uimg_perm); }
   unsigned char *himg_hi() const { return reinterpret_cast<unsigned char *>(tc + T.himg_hi); }
@@ -413,10 +435,93 @@ pi_status run_sets(const pi_ffn *h, const int32_t *idx, const int32_t *count, in
   return PI_OK;
 }
 
+// Test support (pi_debug_wait_fault): an entry of h that is never published,
+// and a shorter limit for every bounded wait of the fused and batch
+// kernels.
+struct WaitFault {
+  int withhold = -1;
+  unsigned long long limit_ns = 0;  // 0: the kernel's default
+};
+WaitFault g_wait_fault;
+
+// ---------------------------------------------------------------- batch kernel (2..8 tokens)
+namespace BK = pi::batch;
+
+// The batch kernel takes fp16 weights with d a multiple of 64 (d <= 12288),
+// 2..8 tokens, and at most kMaxLoc list positions per CTA.
+bool batch_ok(const pi_ffn *h, int B, int G) {
+  const pi_ffn_desc &D = h->d;
+  if (B < 2 || B > BK::kTok || D.wtype != PI_W_F16) return false;
+  if (D.d_model % BK::kTileCols || D.d_model / BK::kTileCols > BK::kMaxTiles) return false;
+  const int nm = D.act == PI_ACT_SWIGLU ? 2 : 1;
+  if (BK::smem_bytes(D.d_model, nm) > 200 * 1024) return false;
+  return (D.d_ffn + G - 1) / G <= BK::kMaxLoc;
+}
+
+template <int ACT>
+cudaError_t batch_launch(const BK::Args &a, int G, int d, cudaStream_t st) {
+  static int attr_smem = 0;
+  const int smem = (int)BK::smem_bytes(d, ACT == pi::ACT_SWIGLU ? 2 : 1);
+  if (smem > attr_smem) {
+    cudaError_t e = cudaFuncSetAttribute(BK::ffn_batch_kernel<ACT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         200 * 1024);
+    if (e != cudaSuccess) return e;
+    attr_smem = 200 * 1024;
+  }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(G);
+  cfg.blockDim = dim3(BK::kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  // programmatic dependent launch, no cooperative attribute: one CTA per SM,
+  // and the one grid-wide wait is bounded (PI_ERR_TIMEOUT, never a hang)
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, BK::ffn_batch_kernel<ACT>, a);
+}
+
+pi_status run_ffn_batch(const pi_ffn *h, const void *u, int B, float *out, int accumulate, unsigned flags,
+                        const Ws &w, cudaStream_t st) {
+  const pi_ffn_desc &D = h->d;
+  BK::Args a{};
+  a.w_up = D.w_up;
+  a.w_gate = D.w_gate;
+  a.w_down_t = D.w_down_t;
+  a.b_up = D.b_up;
+  a.u = reinterpret_cast<const __half *>(u);
+  a.d = D.d_model;
+  a.f = D.d_ffn;
+  a.B = B;
+  a.mask = w.mask();
+  a.nwords = h->nwords;
+  a.ulist = w.ulist();
+  a.ucount = w.ucount();
+  a.uprefix = w.uprefix();
+  a.hot_dense = want_dense(h, B, flags) ? 1 : 0;
+  a.H = h->H;
+  a.a_hi = w.b_ahi();
+  a.a_lo = w.b_alo();
+  a.a_stride = w.L.a_stride;
+  a.part = w.b_part();
+  a.ctr = w.b_ctr();
+  a.bar = w.grid_bar();
+  a.out = out;
+  a.accumulate = accumulate;
+  a.status = w.status();
+  a.wait_ns = g_wait_fault.limit_ns ? g_wait_fault.limit_ns : BK::kWaitNs;
+  const cudaError_t e = D.act == PI_ACT_RELU ? batch_launch<pi::ACT_RELU>(a, w.L.G, D.d_model, st)
+                                             : batch_launch<pi::ACT_SWIGLU>(a, w.L.G, D.d_model, st);
+  return e == cudaSuccess ? PI_OK : PI_ERR_CUDA;
+}
+
 // steps 3-4 over the union in the workspace; out (=, +=) y
 pi_status run_ffn(const pi_ffn *h, const void *u, int B, float *out, int accumulate, unsigned flags, const Ws &w,
                   cudaStream_t st) {
   const pi_ffn_desc &D = h->d;
+  if (batch_ok(h, B, w.L.G)) return run_ffn_batch(h, u, B, out, accumulate, flags, w, st);
   pi::FfnArgs a{};
   a.w_up = D.w_up;
   a.w_gate = D.w_gate;
@@ -609,13 +714,6 @@ pi_status run_ffn_tc(const pi_ffn *h, const void *u, int B, float *out, int accu
 // ---------------------------------------------------------------- fused batch-1 path
 namespace F = pi::fused;
 
-// Test support (pi_debug_wait_fault): an entry of h that is never published,
-// and a shorter limit for every bounded wait of the fused kernel.
-struct WaitFault {
-  int withhold = -1;
-  unsigned long long limit_ns = 0;  // 0: the kernel's default
-};
-WaitFault g_wait_fault;
 
 template <int WT, int ACT, int CPT>
 cudaError_t fused_launch(const F::Args &a, int G, cudaStream_t st) {

@@ -77,7 +77,7 @@ enum ItemType : int { IT_P1 = 0, IT_P2 = 1, IT_GATHER = 2, IT_DONE = 3 };
 
 struct SlotMeta {
   int type, n, first;
-  int tslot;  // gather item of dense hot-prefix rows: slot of their tile's partial scores; else -1
+  int tslot;  // gather item of dense hot-prefix rows: buffer of their tile's partial scores; else -1
   int ids[kMaxGN];
 };
 
@@ -91,7 +91,10 @@ struct Smem {
   float own_pbias[kMaxOwnTiles][kTN];  // predictor bias of this CTA's neurons
   float own_bup[kMaxOwnTiles][kTN];    // ReLU bias b1 of this CTA's neurons
   float h_s[kMaxR];                    // h, gathered from all CTAs
-  float spart[kSlots][kConsumerWarps][kTN];  // per-warp partial scores of the tile in a slot
+  // per-warp partial scores of own tile k, in buffer k % kSlots (tile k + 3
+  // comes at least 3 items after tile k's last dense item, so it is not
+  // issued before every warp is done with that item)
+  float spart[kSlots][kConsumerWarps][kTN];
   float red[2][kConsumerWarps][2 * kMaxGN];
   double dred[kConsumerWarps];
   float fin[kConsumers / (kRedCols / 2)][kRedCols + 1];
@@ -401,7 +404,7 @@ PI_DEV void producer(Smem &S, const Args &a, int c, int G, int lane) {
   // completed: lane q adds the 16 warps' partials of row q in warp order,
   // then the bias; fire iff s > 0
   auto harvest = [&]() {
-    const int s = S.tile_item[hk] % kSlots;
+    const int s = hk % kSlots;
     const int rows = min(kTN, nn - hk * kTN);
     float v = 0.f;
 #pragma unroll
@@ -447,8 +450,9 @@ PI_DEV void producer(Smem &S, const Args &a, int c, int G, int lane) {
     while (hk < k && (unsigned)S.tile_item[hk] + kSlots <= pn) harvest();
     return true;
   };
-  // gather item: own indices ms[0..n); lane j issues copy j.  tslot: slot of
-  // the tile of dense hot-prefix rows (their bits are not known yet), else -1
+  // gather item: own indices ms[0..n); lane j issues copy j.  tslot: buffer
+  // of the partial scores of the tile of dense hot-prefix rows (their bits
+  // are not known yet), else -1
   auto issue_gather = [&](const int *ms, int n, int tslot) -> bool {
     int s;
     if (!acquire(s)) return false;
@@ -536,7 +540,7 @@ PI_DEV void producer(Smem &S, const Args &a, int c, int G, int lane) {
       __syncwarp();
       ++pn;
       // dense hot prefix: the tile's prefix neurons (the smallest ids), now
-      const int ts = (int)((pn - 1) % kSlots);
+      const int ts = k % kSlots;
       int ms[kMaxGN], ng = 0;
       for (int q = 0; ok && q < rows; ++q) {
         if (c + (k * kTN + q) * G >= a.H) break;
@@ -894,11 +898,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
       }
       // lanes 4g hold rows g and g + 8 of each half: s = D[.,0] + D[.,1]
       if ((lane & 3) == 0) {
-        const int g = lane >> 2;
-        S.spart[s][warp][g] = acc[0][0] + acc[0][1];
-        S.spart[s][warp][g + 8] = acc[0][2] + acc[0][3];
-        S.spart[s][warp][g + 16] = acc[1][0] + acc[1][1];
-        S.spart[s][warp][g + 24] = acc[1][2] + acc[1][3];
+        const int g = lane >> 2, b = kl % kSlots;
+        S.spart[b][warp][g] = acc[0][0] + acc[0][1];
+        S.spart[b][warp][g + 8] = acc[0][2] + acc[0][3];
+        S.spart[b][warp][g + 16] = acc[1][0] + acc[1][1];
+        S.spart[b][warp][g + 24] = acc[1][2] + acc[1][3];
       }
       release(s);
       continue;
@@ -906,21 +910,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
     // IT_GATHER: neurons past the item alias neuron 0 and get a zero value.
     // Index-mode items hold fired neurons only; for dense hot-prefix rows the
     // lanes 8g work out membership from their tile's partial scores (same
-    // sum, same order as the producer's), before the barrier below, since the
-    // next tile in that slot may overwrite them once every warp has passed it
+    // sum, same order as the producer's) after the barrier below, when every
+    // warp has written its partials of that tile
     const int ng = S.meta[s].n;
-    bool member = true;
-    {
-      const int ts = S.meta[s].tslot;
-      const int g_l = lane >> 3;
-      if (ts >= 0 && (lane & 7) == 0 && g_l < ng) {
-        const int m = S.meta[s].ids[g_l];
-        float v = 0.f;
-#pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) v += S.spart[ts][w][m % kTN];
-        member = v + S.own_pbias[m / kTN][m % kTN] > 0.f;
-      }
-    }
     const uint8_t *nd[kMaxGN];
 #pragma unroll
     for (int g = 0; g < kMaxGN; ++g) nd[g] = S.ring[s] + (g < ng ? g : 0) * NL.bytes;
@@ -999,6 +991,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
       if ((lane & 7) == 0 && g_l < ng) {
         const int m = S.meta[s].ids[g_l];  // own index: neuron c + m G
         const int kl = m / kTN;
+        bool member = true;
+        const int ts = S.meta[s].tslot;
+        if (ts >= 0) {
+          float v = 0.f;
+#pragma unroll
+          for (int w = 0; w < kConsumerWarps; ++w) v += S.spart[ts][w][m % kTN];
+          member = v + S.own_pbias[kl][m % kTN] > 0.f;
+        }
         if (member) {
           if (ACT == ACT_RELU)
             a_l = fmaxf(vu + S.own_bup[kl][m % kTN], 0.f);

@@ -190,7 +190,7 @@ pi_status pi_decode_ffn_stack(const pi_ffn_t *layers, int L, float *x, int B, in
  *    and, per SM, one fp32 and one tagged 8-byte partial row of d entries)
  *    must fit PI_STATIC_SCRATCH_BYTES; otherwise the call returns
  *    PI_ERR_WORKSPACE and launches nothing.  On a 148-SM B200 this admits
- *    d_model <= 9360 at d_ffn = 28672 and rank 1024, i.e. every OPT-7B- to
+ *    d_model <= 9357 at d_ffn = 28672 and rank 1024, i.e. every OPT-7B- to
  *    LLaMA2-70B-shaped layer (d_model <= 8192).
  *  - The first call on each device (and again after a device reset) does
  *    the set-up: it looks up the array's device address with the device

@@ -200,3 +200,19 @@ def test_full_size_layer(cuda_device, name):
     for B in [b for b in cfg.batches if b <= 8]:
         x = inputs.make_tokens(cfg, 0, B, seed=0)
         check_layer(lt, inputs.layer_input(cfg, x), g)
+
+
+@pytest.mark.parametrize("name,B", [("llama13b_swiglu_f16", 1), ("llama13b_swiglu_f16", 4), ("opt7b_f16", 1),
+                                    ("opt7b_f16", 8)])
+def test_repeated_decode_is_bitwise_stable(cuda_device, name, B):
+    """A full-size layer decoded 200 times on the same tokens gives the same
+    bits every time: sums run in a fixed order, so any difference is a race
+    (a partial read before it is written, a buffer reused too early)."""
+    cfg = inputs.CONFIGS[name]
+    lt = inputs.make_layer(cfg, layer=cfg.n_layers - 1, seed=0, device="cuda")
+    g = Gpu(lt, 8)
+    u = inputs.layer_input(cfg, inputs.make_tokens(cfg, 0, B, seed=0).cuda()).cuda()
+    y0 = g.decode(u)[0].clone()
+    bad = sum(int(not torch.equal(g.decode(u)[0], y0)) for _ in range(200))
+    assert bad == 0, f"{bad} of 200 repeated decodes differ"
+    assert g.status() == 0
