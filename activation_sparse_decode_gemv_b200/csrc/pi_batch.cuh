@@ -13,11 +13,13 @@
 // Step 3 (up / gate + activation).  CTA c takes the list positions
 // [chunk_begin(c), chunk_begin(c + 1)), in groups of 16 neurons (the MMA's M).
 // A unit is 64 elements of the 16 rows of a group.  The weight rows go from
-// HBM straight into registers: lane (g, q) of a warp loads 16 bytes at
-// elements 8q and 32 + 8q of rows g and g + 8, which is an A fragment once the
-// K order inside the unit is permuted the same way for the token operand (a
-// dot product does not depend on the order of its terms).  The tokens sit in
-// shared memory.  The CTA's units are split into 16 contiguous spans, one per
+// HBM straight into registers: lane (g, q) of a warp loads the 32 bytes at
+// elements 16q .. 16q + 15 of rows g and g + 8 (one 256-bit load each, so the
+// four lanes of a row read its whole 128-byte line in one instruction; half
+// lines per instruction were measured to cost HBM more than half its
+// bandwidth).  Those are A fragments once the K order inside the unit is
+// permuted the same way for the token operand (a dot product does not depend
+// on the order of its terms).  The tokens sit in shared memory.  The CTA's units are split into 16 contiguous spans, one per
 // warp (stream-K inside the CTA); each warp leaves one partial per group it
 // touched in shared memory and the CTA adds them in warp order.  The
 // activation a (zero for tokens that did not predict the neuron) is stored as
@@ -88,7 +90,7 @@ struct Args {
 // dynamic shared memory: step 3 (tokens + warp partials) and step 4 (stages +
 // tile partials) use the same bytes, one after the other
 inline __host__ __device__ size_t step3_bytes(int d, int nmat) {
-  return (size_t)kTok * (2 * (size_t)d + 64) + (size_t)kWarps * kMaxSlots * nmat * 128 * 4;
+  return (size_t)kTok * (2 * (size_t)d + 16) + (size_t)kWarps * kMaxSlots * nmat * 128 * 4;
 }
 inline __host__ __device__ size_t step4_bytes() {
   return (size_t)kWarps * kStages * kStageBytes + (size_t)kWarps * kPieceFloats * 4;
@@ -103,6 +105,12 @@ PI_DEV void ldmatrix_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                : "r"(addr));
+}
+// 32 bytes (32-byte aligned) of a weight row, read once: bypass L1
+PI_DEV void ld_stream32(const void *p, uint4 &lo, uint4 &hi) {
+  asm("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+      : "=r"(lo.x), "=r"(lo.y), "=r"(lo.z), "=r"(lo.w), "=r"(hi.x), "=r"(hi.y), "=r"(hi.z), "=r"(hi.w)
+      : "l"(p));
 }
 PI_DEV void cp_async16(uint32_t dst, const void *src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
@@ -138,6 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
   __shared__ uint32_t memb_s[kMaxLoc];
   __shared__ float bias_s[kMaxLoc];
   __shared__ int last_s;
+  __shared__ int span_lo_s[kWarps], span_jlo_s[kWarps], span_jhi_s[kWarps];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, q = lane & 3;
   const int G = gridDim.x, c = blockIdx.x;
   const int d = a.d, B = a.B;
@@ -151,7 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
   // ================================================================ step 3
   const int pb = list_begin(c, V, G), pe = list_begin(c + 1, V, G);
   const int nloc = pe - pb;
-  const int upitch = d + 32;  // halves; rows 64 bytes apart modulo 128
+  const int upitch = d + 8;  // halves; rows 16 bytes apart modulo 128 (conflict-free fragment reads)
   __half *u_s = reinterpret_cast<__half *>(smem);
   float *red = reinterpret_cast<float *>(smem + (size_t)kTok * upitch * 2);
   {
@@ -176,33 +185,33 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
   const int ns = d / kKStep;
   const int ng = (nloc + 15) >> 4;
   const int T = ng * ns;
-  const int w0 = (int)((long long)T * warp / kWarps), w1 = (int)((long long)T * (warp + 1) / kWarps);
+  const int w0 = T * warp / kWarps, w1 = T * (warp + 1) / kWarps;
   const int ja = w0 / ns;
+  if (tid < kWarps) {  // each warp's span, for the reduction (T * 16 < 2^31)
+    const int lo = T * tid / kWarps, hi = T * (tid + 1) / kWarps;
+    span_lo_s[tid] = lo < hi ? 1 : 0;
+    span_jlo_s[tid] = lo / ns;
+    span_jhi_s[tid] = lo < hi ? (hi - 1) / ns : -1;
+  }
   {
     struct Buf {
-      uint4 w[NM][4];  // [matrix][row g lo, row g hi, row g+8 lo, row g+8 hi]
+      uint4 w[NM][4];  // [matrix][row g elements 0-7, 8-15, row g+8 elements 0-7, 8-15] of this lane's 16
     };
     auto load = [&](Buf &bf, int ui) {
       const int j = ui / ns, s = ui - j * ns;
       const int r0 = 16 * j + g, r1 = r0 + 8;
-      const size_t off = (size_t)s * (kKStep * 2) + (size_t)q * 16;
+      const size_t off = (size_t)s * (kKStep * 2) + (size_t)q * 32;
 #pragma unroll
       for (int m = 0; m < NM; ++m) {
         const char *W = reinterpret_cast<const char *>(m == 0 ? a.w_up : a.w_gate);
-        if (r0 < nloc) {
-          const char *p = W + (size_t)ids_s[r0] * rb + off;
-          bf.w[m][0] = ld_stream16(p);
-          bf.w[m][1] = ld_stream16(p + 64);
-        } else {
+        if (r0 < nloc)
+          ld_stream32(W + (size_t)ids_s[r0] * rb + off, bf.w[m][0], bf.w[m][1]);
+        else
           bf.w[m][0] = bf.w[m][1] = make_uint4(0u, 0u, 0u, 0u);
-        }
-        if (r1 < nloc) {
-          const char *p = W + (size_t)ids_s[r1] * rb + off;
-          bf.w[m][2] = ld_stream16(p);
-          bf.w[m][3] = ld_stream16(p + 64);
-        } else {
+        if (r1 < nloc)
+          ld_stream32(W + (size_t)ids_s[r1] * rb + off, bf.w[m][2], bf.w[m][3]);
+        else
           bf.w[m][2] = bf.w[m][3] = make_uint4(0u, 0u, 0u, 0u);
-        }
       }
     };
     float acc[NM][4];
@@ -212,8 +221,9 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
       for (int e = 0; e < 4; ++e) acc[m][e] = 0.f;
     auto compute = [&](const Buf &bf, int ui) {
       const int j = ui / ns, s = ui - j * ns;
-      const __half *ur = u_s + (size_t)g * upitch + (size_t)s * kKStep + q * 8;
-      const uint4 ub0 = *reinterpret_cast<const uint4 *>(ur), ub1 = *reinterpret_cast<const uint4 *>(ur + 32);
+      // token g's elements 16q .. 16q + 15 of the unit, the same K order as the rows
+      const __half *ur = u_s + (size_t)g * upitch + (size_t)s * kKStep + q * 16;
+      const uint4 ub0 = *reinterpret_cast<const uint4 *>(ur), ub1 = *reinterpret_cast<const uint4 *>(ur + 8);
 #pragma unroll
       for (int m = 0; m < NM; ++m) {
         const uint4 &x0 = bf.w[m][0], &x1 = bf.w[m][1], &y0 = bf.w[m][2], &y1 = bf.w[m][3];
@@ -270,10 +280,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
 #pragma unroll
     for (int m = 0; m < NM; ++m) x[m] = 0.f;
     for (int w = 0; w < kWarps; ++w) {
-      const int lo = (int)((long long)T * w / kWarps), hi = (int)((long long)T * (w + 1) / kWarps);
-      if (lo >= hi) continue;
-      const int jlo = lo / ns, jhi = (hi - 1) / ns;
-      if (j < jlo || j > jhi) continue;
+      const int jlo = span_jlo_s[w];
+      if (!span_lo_s[w] || j < jlo || j > span_jhi_s[w]) continue;
 #pragma unroll
       for (int m = 0; m < NM; ++m) x[m] += red[(size_t)((w * kMaxSlots + (j - jlo)) * NM + m) * 128 + ln * 4 + e];
     }
@@ -342,7 +350,20 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
     const __half *src = (hl ? a.a_lo : a.a_hi) + (size_t)t8 * a.a_stride + (size_t)s * kPosStep + half * 8;
     cp_async16(st + (uint32_t)(kPosStep * kRowBytes + hl * (kTok * kPosStep * 2) + t8 * 32 + half * 16), src);
   };
-  auto issue = [&](int k, bool rows, bool acts) {
+  // list ids of the rows this lane copies for unit k (rows lane / 8 + 4 i),
+  // fetched one unit ahead so the copies do not wait for them
+  auto fetch_ids = [&](int k, int (&id)[4]) {
+    if (k < K) {
+      int t, s;
+      unit_of(k, t, s);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int p = s * kPosStep + (lane >> 3) + 4 * i;
+        id[i] = p < V ? vid(p) : -1;
+      }
+    }
+  };
+  auto issue = [&](int k, const int (&id)[4], bool rows, bool acts) {
     if (k < K) {
       int t, s;
       unit_of(k, t, s);
@@ -351,10 +372,9 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int row = (lane >> 3) + 4 * i, ch = lane & 7;
-          const int p = s * kPosStep + row;
           const uint32_t dst = st + (uint32_t)(row * kRowBytes + ((ch ^ (row & 7)) << 4));
-          if (p < V)
-            cp_async16(dst, Wd + (size_t)vid(p) * rb + (size_t)t * kRowBytes + ch * 16);
+          if (id[i] >= 0)
+            cp_async16(dst, Wd + (size_t)id[i] * rb + (size_t)t * kRowBytes + ch * 16);
           else
             st_shared_zero16(dst);
         }
@@ -366,8 +386,13 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
 
   // the first stages' weight rows do not depend on step 3: in flight during
   // the grid-wide wait
+  int ids_next[4];
 #pragma unroll
-  for (int k = 0; k < kStages - 1; ++k) issue(k, true, false);
+  for (int k = 0; k < kStages - 1; ++k) {
+    fetch_ids(k, ids_next);
+    issue(k, ids_next, true, false);
+  }
+  fetch_ids(kStages - 1, ids_next);
   if (tid == 0) grid_barrier(a.bar, G, c, a.status, a.wait_ns);
   __syncthreads();
   pdl_launch_dependents();
@@ -415,7 +440,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
         mma_16816(acc_l[mt], A, bl0, bl1);
       }
       __syncwarp();
-      issue(k + kStages - 1, true, true);
+      issue(k + kStages - 1, ids_next, true, true);
+      fetch_ids(k + kStages, ids_next);
     }
     // this warp's partial of tile t
 #pragma unroll

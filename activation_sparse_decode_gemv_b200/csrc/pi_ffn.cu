@@ -448,10 +448,13 @@ WaitFault g_wait_fault;
 namespace BK = pi::batch;
 
 // The batch kernel takes fp16 weights with d a multiple of 64 (d <= 12288),
-// 2..8 tokens, and at most kMaxLoc list positions per CTA.
+// up / gate matrices on 32-byte boundaries (256-bit row loads), 2..8 tokens,
+// and at most kMaxLoc list positions per CTA.
 bool batch_ok(const pi_ffn *h, int B, int G) {
   const pi_ffn_desc &D = h->d;
   if (B < 2 || B > BK::kTok || D.wtype != PI_W_F16) return false;
+  if ((reinterpret_cast<uintptr_t>(D.w_up) & 31u) || (D.w_gate && (reinterpret_cast<uintptr_t>(D.w_gate) & 31u)))
+    return false;
   if (D.d_model % BK::kTileCols || D.d_model / BK::kTileCols > BK::kMaxTiles) return false;
   const int nm = D.act == PI_ACT_SWIGLU ? 2 : 1;
   if (BK::smem_bytes(D.d_model, nm) > 200 * 1024) return false;
