@@ -498,5 +498,185 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
   cp_async_wait<0>();
 }
 
+
+// ================================================================ predictor (batches of 2..8)
+// The same tensor-core row dot as step 3: weight rows as A fragments loaded
+// with 256-bit loads (elements 16q .. 16q + 15 of a 64-element unit per
+// lane), the tokens (or h) as the B operand in the matching K order.  The
+// weight rows do not depend on the previous kernel, so each kernel loads its
+// rows into registers before griddepcontrol.wait: P2 streams in while P1 is
+// still being reduced.
+struct PredArgs {
+  const __half *p1, *p2;
+  const float *p_bias;
+  const __half *u;  // [B x d]
+  float *h;         // [B x r]
+  int d, r, f, B;
+  uint32_t *mask;    // [B x nwords]
+  uint32_t *uwords;  // [nwords], OR of the tokens' words
+  int nwords;
+};
+constexpr int kPredHRows = 8;   // P1 rows per CTA (MMA rows 0..7; rows 8..15 are zero)
+constexpr int kPredHUnits = 8;  // 64-element units per warp (d <= 8192)
+constexpr int kPredSWarps = 8;  // pred_s: 2 groups of 16 rows x 4 quarters of the rank
+constexpr int kPredSUnits = 4;  // units per warp (rank <= 1024)
+
+PI_DEV uint4 ld_cg16(const void *p) {
+  uint4 v;
+  asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
+}
+PI_DEV float4 ld_cg_f4(const float *p) {
+  float4 v;
+  asm volatile("ld.global.cg.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(p));
+  return v;
+}
+
+// h[t][j] = P1_j . u_t for the 8 rows j of CTA blockIdx.x; warp w takes the
+// units [w ns / 16, (w + 1) ns / 16) of the d / 64 units, the CTA adds the
+// warps' partials in warp order.
+__global__ void __launch_bounds__(kThreads) pred_h_batch_kernel(const __grid_constant__ PredArgs a) {
+  __shared__ float red[kWarps][64];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, q = lane & 3;
+  const int d = a.d, r = a.r;
+  const int j = blockIdx.x * kPredHRows + g;
+  const int ns = d / kKStep;
+  const int w0 = ns * warp / kWarps, w1 = ns * (warp + 1) / kWarps;
+  uint4 wl[kPredHUnits], wh[kPredHUnits];
+#pragma unroll
+  for (int i = 0; i < kPredHUnits; ++i) {
+    wl[i] = wh[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (w0 + i < w1 && j < r) ld_stream32(a.p1 + (size_t)j * d + (size_t)(w0 + i) * kKStep + q * 16, wl[i], wh[i]);
+  }
+  pdl_wait();
+  pdl_launch_dependents();
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int i = 0; i < kPredHUnits; ++i) {
+    if (w0 + i < w1) {
+      uint4 ub0 = make_uint4(0u, 0u, 0u, 0u), ub1 = ub0;
+      if (g < a.B) {
+        const __half *up = a.u + (size_t)g * d + (size_t)(w0 + i) * kKStep + q * 16;
+        ub0 = ld_cg16(up);
+        ub1 = ld_cg16(up + 8);
+      }
+      const uint4 &x0 = wl[i], &x1 = wh[i];
+      {
+        const uint32_t A[4] = {x0.x, 0u, x0.y, 0u};
+        mma_16816(acc, A, ub0.x, ub0.y);
+      }
+      {
+        const uint32_t A[4] = {x0.z, 0u, x0.w, 0u};
+        mma_16816(acc, A, ub0.z, ub0.w);
+      }
+      {
+        const uint32_t A[4] = {x1.x, 0u, x1.y, 0u};
+        mma_16816(acc, A, ub1.x, ub1.y);
+      }
+      {
+        const uint32_t A[4] = {x1.z, 0u, x1.w, 0u};
+        mma_16816(acc, A, ub1.z, ub1.w);
+      }
+    }
+  }
+  // lane (g, q) holds row g, tokens 2q and 2q + 1
+  red[warp][lane * 2] = acc[0];
+  red[warp][lane * 2 + 1] = acc[1];
+  __syncthreads();
+  if (tid < kPredHRows * kTok) {
+    const int row = tid >> 3, t = tid & 7;
+    const int jr = blockIdx.x * kPredHRows + row;
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) v += red[w][(row * 4 + (t >> 1)) * 2 + (t & 1)];
+    if (t < a.B && jr < r) a.h[(size_t)t * r + jr] = v;
+  }
+}
+
+// s_i = P2_i . h + bias_i and the fired bits for the 32 rows of CTA
+// blockIdx.x (one mask word per token).  Warp w: group w & 1 (16 rows),
+// quarter w >> 1 of the rank; B operand = h split into fp16 h_hi and
+// h_lo = fp16(h - h_hi), as two MMAs, so h enters with about 22 bits.
+__global__ void __launch_bounds__(kPredSWarps * 32) pred_s_batch_kernel(const __grid_constant__ PredArgs a) {
+  __shared__ float red[kPredSWarps][128];
+  __shared__ uint32_t uw_s[kTok];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, q = lane & 3;
+  const int r = a.r, f = a.f;
+  const int grp = warp & 1, qr = warp >> 1;
+  const int i0 = blockIdx.x * 32 + 16 * grp + g, i1 = i0 + 8;
+  const int nsr = r / kKStep;
+  const int u0 = nsr * qr / 4, u1 = nsr * (qr + 1) / 4;
+  uint4 a0l[kPredSUnits], a0h[kPredSUnits], a1l[kPredSUnits], a1h[kPredSUnits];
+#pragma unroll
+  for (int i = 0; i < kPredSUnits; ++i) {
+    a0l[i] = a0h[i] = a1l[i] = a1h[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (u0 + i < u1) {
+      const size_t off = (size_t)(u0 + i) * kKStep + q * 16;
+      if (i0 < f) ld_stream32(a.p2 + (size_t)i0 * r + off, a0l[i], a0h[i]);
+      if (i1 < f) ld_stream32(a.p2 + (size_t)i1 * r + off, a1l[i], a1h[i]);
+    }
+  }
+  pdl_wait();
+  pdl_launch_dependents();
+  float acc_h[4] = {0.f, 0.f, 0.f, 0.f}, acc_l[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int i = 0; i < kPredSUnits; ++i) {
+    if (u0 + i < u1) {
+      // token g's h at the unit's elements 16q .. 16q + 15, as fp16 hi / lo pairs
+      uint32_t hh[8], hl[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) hh[e] = hl[e] = 0u;
+      if (g < a.B) {
+        const float *hp = a.h + (size_t)g * r + (size_t)(u0 + i) * kKStep + q * 16;
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4) {
+          const float4 x = ld_cg_f4(hp + 4 * v4);
+          hh[2 * v4] = fused::h_part_pair(x.x, x.y, 0);
+          hl[2 * v4] = fused::h_part_pair(x.x, x.y, 1);
+          hh[2 * v4 + 1] = fused::h_part_pair(x.z, x.w, 0);
+          hl[2 * v4 + 1] = fused::h_part_pair(x.z, x.w, 1);
+        }
+      }
+      const uint4 &x0 = a0l[i], &x1 = a0h[i], &y0 = a1l[i], &y1 = a1h[i];
+      const uint32_t A0[4] = {x0.x, y0.x, x0.y, y0.y}, A1[4] = {x0.z, y0.z, x0.w, y0.w};
+      const uint32_t A2[4] = {x1.x, y1.x, x1.y, y1.y}, A3[4] = {x1.z, y1.z, x1.w, y1.w};
+      mma_16816(acc_h, A0, hh[0], hh[1]);
+      mma_16816(acc_l, A0, hl[0], hl[1]);
+      mma_16816(acc_h, A1, hh[2], hh[3]);
+      mma_16816(acc_l, A1, hl[2], hl[3]);
+      mma_16816(acc_h, A2, hh[4], hh[5]);
+      mma_16816(acc_l, A2, hl[4], hl[5]);
+      mma_16816(acc_h, A3, hh[6], hh[7]);
+      mma_16816(acc_l, A3, hl[6], hl[7]);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) red[warp][lane * 4 + e] = acc_h[e] + acc_l[e];
+  if (tid < kTok) uw_s[tid] = 0u;
+  __syncthreads();
+  // warp t: token t, lane = row of the word (group lane >> 4, M row lane & 15)
+  {
+    const int t = warp, row = lane, gr = row >> 4, m = row & 15;
+    const int ln = (m & 7) * 4 + (t >> 1), e = (t & 1) + ((m >> 3) << 1);
+    const int i = blockIdx.x * 32 + row;
+    float s = 0.f;
+#pragma unroll
+    for (int qq = 0; qq < 4; ++qq) s += red[2 * qq + gr][ln * 4 + e];
+    const bool fire = t < a.B && i < f && s + a.p_bias[i < f ? i : 0] > 0.f;
+    const uint32_t bits = __ballot_sync(0xffffffffu, fire);
+    if (lane == 0) {
+      if (t < a.B) a.mask[(size_t)t * a.nwords + blockIdx.x] = bits;
+      uw_s[t] = bits;
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    uint32_t u = 0u;
+#pragma unroll
+    for (int t = 0; t < kTok; ++t) u |= uw_s[t];
+    a.uwords[blockIdx.x] = u;
+  }
+}
+
 }  // namespace batch
 }  // namespace pi

@@ -384,10 +384,42 @@ bool want_dense(const pi_ffn *h, int B, unsigned flags) {
     if ((call) != cudaSuccess) return PI_ERR_CUDA; \
   } while (0)
 
+// The tensor-core predictor kernels of batches 2..8: fp16 predictor, rank a
+// multiple of 64 up to 1024, d a multiple of 64 up to 8192, P1 and P2 on
+// 32-byte boundaries (256-bit row loads).
+bool pred_batch_ok(const pi_ffn *h, int B) {
+  const pi_ffn_desc &D = h->d;
+  if (B < 2 || B > pi::batch::kTok || D.ptype != PI_W_F16) return false;
+  if (D.rank % 64 || D.rank > 64 * 4 * pi::batch::kPredSUnits) return false;
+  if (D.d_model % 64 || D.d_model > 64 * pi::batch::kWarps * pi::batch::kPredHUnits) return false;
+  return !((reinterpret_cast<uintptr_t>(D.p1) | reinterpret_cast<uintptr_t>(D.p2)) & 31u);
+}
+
 // steps 1-2: predictor, mask words, compaction (idx/count optional)
 pi_status run_predict(const pi_ffn *h, const void *u, int B, int32_t *idx, int idx_stride, int32_t *count, const Ws &w,
                       cudaStream_t st) {
   const pi_ffn_desc &D = h->d;
+  if (pred_batch_ok(h, B)) {
+    pi::batch::PredArgs a{};
+    a.p1 = reinterpret_cast<const __half *>(D.p1);
+    a.p2 = reinterpret_cast<const __half *>(D.p2);
+    a.p_bias = D.p_bias;
+    a.u = reinterpret_cast<const __half *>(u);
+    a.h = w.h();
+    a.d = D.d_model;
+    a.r = D.rank;
+    a.f = D.d_ffn;
+    a.B = B;
+    a.mask = w.mask();
+    a.uwords = w.uwords();
+    a.nwords = h->nwords;
+    PI_CUDA(launch(pi::batch::pred_h_batch_kernel, dim3(cdiv(D.rank, pi::batch::kPredHRows)),
+                   dim3(pi::batch::kThreads), st, a));
+    PI_CUDA(launch(pi::batch::pred_s_batch_kernel, dim3(h->nwords), dim3(pi::batch::kPredSWarps * 32), st, a));
+    PI_CUDA(launch(pi::compact_kernel, dim3(B + 1), dim3(1024), st, (const uint32_t *)w.mask(), h->nwords, idx_stride,
+                   B, idx, count, w.uwords(), w.uprefix(), w.ulist(), w.ucount()));
+    return PI_OK;
+  }
   const int nb = nb_for(B);
   const dim3 gh(cdiv(D.rank, 8), cdiv(B, nb)), gs(h->nwords, cdiv(B, nb));
   cudaError_t e;
