@@ -64,6 +64,7 @@ constexpr int kStageBytes = kPosStep * kRowBytes + 2 * kTok * kPosStep * 2;  // 
 constexpr int kMaxLoc = 512;     // list positions one CTA takes in step 3
 constexpr int kMaxSlots = 3;     // groups one warp's step-3 span touches (kMaxLoc / 16 <= 32 groups)
 constexpr int kMaxTiles = 192;   // step-4 tiles (d <= 12288)
+constexpr int kMaxWords = 1024;  // 32-neuron words of the union (d_ffn <= 32768)
 constexpr int kPieceFloats = kTileCols * kTok;
 constexpr unsigned long long kWaitNs = 2000000000ull;
 
@@ -72,9 +73,10 @@ struct Args {
   const float *b_up;
   const __half *u;  // [B x d] fp16
   int d, f, B;
-  const uint32_t *mask;  // [B x nwords] per-token mask words
+  const uint32_t *mask;    // [B x nwords] per-token mask words
+  const uint32_t *uwords;  // [nwords] their OR (the union)
   int nwords;
-  const int32_t *ulist, *ucount, *uprefix;
+  int32_t *ulist;  // union list, written here: each CTA its own positions
   int hot_dense, H;
   __half *a_hi, *a_lo;  // [kTok x a_stride] activations by list position
   int a_stride;
@@ -120,16 +122,22 @@ template <int N>
 PI_DEV void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
+PI_DEV int ld_cg_i32(const int32_t *p) {
+  int v;
+  asm volatile("ld.global.cg.s32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+// position of the k-th (0-based) set bit of w (k < popc(w))
+PI_DEV int select_bit(uint32_t w, int k) {
+  for (int i = 0; i < k; ++i) w &= w - 1u;
+  return __ffs(w) - 1;
+}
 PI_DEV void st_shared_zero16(uint32_t dst) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
 }
 
-// number of list positions of the grid's list and the range of CTA c (the
-// same formulas as the CUDA-core gather kernel)
-PI_DEV int list_len(const int32_t *ucount, const int32_t *uprefix, int hot_dense, int H) {
-  const int U = *ucount;
-  return hot_dense ? H + (U - uprefix[H >> 5]) : U;
-}
+// range of list positions of CTA c (the same formula as the CUDA-core gather
+// kernel)
 PI_DEV int list_begin(int c, int V, int G) { return (int)(((long long)c * V) / G); }
 
 // step-4 span of CTA c: units [span_lo(c), span_lo(c + 1)) of W
@@ -147,15 +155,110 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
   __shared__ float bias_s[kMaxLoc];
   __shared__ int last_s;
   __shared__ int span_lo_s[kWarps], span_jlo_s[kWarps], span_jhi_s[kWarps];
+  __shared__ uint32_t uw_s[kMaxWords];
+  __shared__ int pre_s[kMaxWords + 1];  // exclusive prefix of the union words' popcounts
+  __shared__ int wsum_s[kWarps];
+  __shared__ int pro_ids_s[kWarps][kStages][kPosStep];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, q = lane & 3;
   const int G = gridDim.x, c = blockIdx.x;
   const int d = a.d, B = a.B;
   const size_t rb = (size_t)d * 2;
 
   pdl_wait();
-  const int V = list_len(a.ucount, a.uprefix, a.hot_dense, a.H);
-  const int upre_h = a.hot_dense ? a.uprefix[a.H >> 5] : 0;
-  auto vid = [&](int p) -> int { return a.hot_dense ? (p < a.H ? p : a.ulist[upre_h + (p - a.H)]) : a.ulist[p]; };
+  // ---- the union: every CTA scans the union words itself (same result in
+  // every CTA), so no separate compaction runs before this kernel
+  const int nw = a.nwords;
+  {
+    uint32_t w0 = 0u, w1 = 0u;
+    if (2 * tid < nw) w0 = a.uwords[2 * tid];
+    if (2 * tid + 1 < nw) w1 = a.uwords[2 * tid + 1];
+    if (2 * tid < nw) uw_s[2 * tid] = w0;
+    if (2 * tid + 1 < nw) uw_s[2 * tid + 1] = w1;
+    const int c0 = __popc(w0), cnt = c0 + __popc(w1);
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) wsum_s[warp] = incl;
+    __syncthreads();
+    int base = 0;
+    for (int w = 0; w < warp; ++w) base += wsum_s[w];
+    const int ex = base + incl - cnt;
+    if (2 * tid < nw) pre_s[2 * tid] = ex;
+    if (2 * tid + 1 < nw) pre_s[2 * tid + 1] = ex + c0;
+    if (tid == kThreads - 1) pre_s[nw] = base + incl;
+    __syncthreads();
+  }
+  const int U = pre_s[nw];
+  const int upre_h = a.hot_dense ? pre_s[a.H >> 5] : 0;
+  const int V = a.hot_dense ? a.H + (U - upre_h) : U;
+  // union index of list position p (-1: a dense hot-prefix row, id p)
+  auto uidx = [&](int p) -> int { return a.hot_dense ? (p < a.H ? -1 : upre_h + (p - a.H)) : p; };
+  // neuron id of union index x, from the scan: binary search, then the bit
+  auto id_of_uidx = [&](int x) -> int {
+    int lo = 0, hi = nw;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (pre_s[mid] <= x) lo = mid; else hi = mid;
+    }
+    return lo * 32 + select_bit(uw_s[lo], x - pre_s[lo]);
+  };
+  auto vid_local = [&](int p) -> int {
+    const int x = uidx(p);
+    return x < 0 ? p : id_of_uidx(x);
+  };
+  // after the grid-wide wait: the list written by the CTAs in step 3
+  auto vid = [&](int p) -> int {
+    const int x = uidx(p);
+    return x < 0 ? p : ld_cg_i32(a.ulist + x);
+  };
+
+  // ---- step-4 spans (known once the list length is): CTA c owns units
+  // [u0, u1) of the W = (d / 64) x S (tile, 16-position step) units
+  const int ntiles = d / kTileCols;
+  const int S = (V + kPosStep - 1) / kPosStep;
+  const long long W = (long long)ntiles * S;
+  const long long u0 = span_lo(W, c, G), u1 = span_lo(W, c + 1, G);
+  const int ta = u0 < u1 ? (int)(u0 / S) : 0, tb = u0 < u1 ? (int)((u1 - 1) / S) : -1;
+  // units of tile t in this CTA's span: steps [sa, sb)
+  auto tile_steps = [&](int t, int &sa, int &sb) {
+    const long long lo = (long long)t * S, hi = lo + S;
+    sa = (int)((u0 > lo ? u0 : lo) - lo);
+    sb = (int)((u1 < hi ? u1 : hi) - lo);
+  };
+  // warp w takes the steps sa + w, sa + w + 16, ... of each tile
+  auto warp_count = [&](int t, int w) {
+    int sa, sb;
+    tile_steps(t, sa, sb);
+    return sb - sa > w ? (sb - sa - w + kWarps - 1) / kWarps : 0;
+  };
+  // k-th unit of warp w -> (tile, step); false past its last unit
+  auto unit_of_w = [&](int k, int w, int &t, int &s) -> bool {
+    for (t = ta; t <= tb; ++t) {
+      const int n = warp_count(t, w);
+      if (k < n) {
+        int sa, sb;
+        tile_steps(t, sa, sb);
+        s = sa + w + k * kWarps;
+        return true;
+      }
+      k -= n;
+    }
+    return false;
+  };
+  // list ids of the first kStages units of every warp (the ones issued before
+  // the grid-wide wait, when the list written in step 3 is not complete)
+  for (int e = tid; e < kWarps * kStages * kPosStep; e += kThreads) {
+    const int w = e / (kStages * kPosStep), k = (e / kPosStep) % kStages, row = e % kPosStep;
+    int t, s, id = -1;
+    if (unit_of_w(k, w, t, s)) {
+      const int p = s * kPosStep + row;
+      if (p < V) id = vid_local(p);
+    }
+    pro_ids_s[w][k][row] = id;
+  }
 
   // ================================================================ step 3
   const int pb = list_begin(c, V, G), pe = list_begin(c + 1, V, G);
@@ -172,7 +275,9 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
       *reinterpret_cast<uint4 *>(u_s + (size_t)t * upitch + (size_t)e * 8) = v;
     }
     for (int k = tid; k < nloc; k += kThreads) {
-      const int i = vid(pb + k);
+      const int x = uidx(pb + k);
+      const int i = x < 0 ? pb + k : id_of_uidx(x);
+      if (x >= 0) a.ulist[x] = i;
       uint32_t m = 0u;
       for (int t = 0; t < B; ++t) m |= ((a.mask[(size_t)t * a.nwords + (i >> 5)] >> (i & 31)) & 1u) << t;
       ids_s[k] = i;
@@ -308,40 +413,12 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
   __syncthreads();
 
   // ================================================================ step 4
-  const int ntiles = d / kTileCols;
-  const int S = (V + kPosStep - 1) / kPosStep;
-  const long long W = (long long)ntiles * S;
-  const long long u0 = span_lo(W, c, G), u1 = span_lo(W, c + 1, G);
   const uint32_t ring = smem_u32(smem) + (uint32_t)(warp * kStages * kStageBytes);
   float *tred = reinterpret_cast<float *>(smem + (size_t)kWarps * kStages * kStageBytes);
   const char *Wd = reinterpret_cast<const char *>(a.w_down_t);
-  const int ta = u0 < u1 ? (int)(u0 / S) : 0, tb = u0 < u1 ? (int)((u1 - 1) / S) : -1;
-  // units of tile t in this CTA's span: steps [sa, sb)
-  auto tile_steps = [&](int t, int &sa, int &sb) {
-    const long long lo = (long long)t * S, hi = lo + S;
-    sa = (int)((u0 > lo ? u0 : lo) - lo);
-    sb = (int)((u1 < hi ? u1 : hi) - lo);
-  };
-  auto warp_count = [&](int t) {
-    int sa, sb;
-    tile_steps(t, sa, sb);
-    return sb - sa > warp ? (sb - sa - warp + kWarps - 1) / kWarps : 0;
-  };
   int K = 0;
-  for (int t = ta; t <= tb; ++t) K += warp_count(t);
-  // k-th unit of this warp -> (tile, step)
-  auto unit_of = [&](int k, int &t, int &s) {
-    for (t = ta; t <= tb; ++t) {
-      const int n = warp_count(t);
-      if (k < n) {
-        int sa, sb;
-        tile_steps(t, sa, sb);
-        s = sa + warp + k * kWarps;
-        return;
-      }
-      k -= n;
-    }
-  };
+  for (int t = ta; t <= tb; ++t) K += warp_count(t, warp);
+  auto unit_of = [&](int k, int &t, int &s) { unit_of_w(k, warp, t, s); };
   auto issue_acts = [&](int k) {
     int t, s;
     unit_of(k, t, s);
@@ -352,14 +429,14 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
   };
   // list ids of the rows this lane copies for unit k (rows lane / 8 + 4 i),
   // fetched one unit ahead so the copies do not wait for them
-  auto fetch_ids = [&](int k, int (&id)[4]) {
+  auto fetch_ids = [&](int k, int (&id)[4], bool local) {
     if (k < K) {
       int t, s;
       unit_of(k, t, s);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const int p = s * kPosStep + (lane >> 3) + 4 * i;
-        id[i] = p < V ? vid(p) : -1;
+        const int row = (lane >> 3) + 4 * i, p = s * kPosStep + row;
+        id[i] = local ? pro_ids_s[warp][k][row] : (p < V ? vid(p) : -1);
       }
     }
   };
@@ -389,10 +466,10 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
   int ids_next[4];
 #pragma unroll
   for (int k = 0; k < kStages - 1; ++k) {
-    fetch_ids(k, ids_next);
+    fetch_ids(k, ids_next, true);
     issue(k, ids_next, true, false);
   }
-  fetch_ids(kStages - 1, ids_next);
+  fetch_ids(kStages - 1, ids_next, true);
   if (tid == 0) grid_barrier(a.bar, G, c, a.status, a.wait_ns);
   __syncthreads();
   pdl_launch_dependents();
@@ -414,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
     for (int e = 0; e < 4; ++e) acc_h[mt][e] = acc_l[mt][e] = 0.f;
   int k = 0;
   for (int t = ta; t <= tb; ++t) {
-    const int nt = warp_count(t);
+    const int nt = warp_count(t, warp);
     for (int n = 0; n < nt; ++n, ++k) {
       if (k == 0)
         cp_async_wait<0>();
@@ -441,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
       }
       __syncwarp();
       issue(k + kStages - 1, ids_next, true, true);
-      fetch_ids(k + kStages, ids_next);
+      fetch_ids(k + kStages, ids_next, false);
     }
     // this warp's partial of tile t
 #pragma unroll

@@ -395,7 +395,10 @@ bool pred_batch_ok(const pi_ffn *h, int B) {
   return !((reinterpret_cast<uintptr_t>(D.p1) | reinterpret_cast<uintptr_t>(D.p2)) & 31u);
 }
 
-// steps 1-2: predictor, mask words, compaction (idx/count optional)
+bool batch_ok(const pi_ffn *h, int B, int G);
+
+// steps 1-2: predictor, mask words, compaction (idx/count optional; the batch
+// FFN kernel scans the union words itself, so without lists it needs none)
 pi_status run_predict(const pi_ffn *h, const void *u, int B, int32_t *idx, int idx_stride, int32_t *count, const Ws &w,
                       cudaStream_t st) {
   const pi_ffn_desc &D = h->d;
@@ -416,8 +419,9 @@ pi_status run_predict(const pi_ffn *h, const void *u, int B, int32_t *idx, int i
     PI_CUDA(launch(pi::batch::pred_h_batch_kernel, dim3(cdiv(D.rank, pi::batch::kPredHRows)),
                    dim3(pi::batch::kThreads), st, a));
     PI_CUDA(launch(pi::batch::pred_s_batch_kernel, dim3(h->nwords), dim3(pi::batch::kPredSWarps * 32), st, a));
-    PI_CUDA(launch(pi::compact_kernel, dim3(B + 1), dim3(1024), st, (const uint32_t *)w.mask(), h->nwords, idx_stride,
-                   B, idx, count, w.uwords(), w.uprefix(), w.ulist(), w.ucount()));
+    if (idx || count || !batch_ok(h, B, w.L.G))
+      PI_CUDA(launch(pi::compact_kernel, dim3(B + 1), dim3(1024), st, (const uint32_t *)w.mask(), h->nwords,
+                     idx_stride, B, idx, count, w.uwords(), w.uprefix(), w.ulist(), w.ucount()));
     return PI_OK;
   }
   const int nb = nb_for(B);
@@ -488,6 +492,7 @@ bool batch_ok(const pi_ffn *h, int B, int G) {
   if ((reinterpret_cast<uintptr_t>(D.w_up) & 31u) || (D.w_gate && (reinterpret_cast<uintptr_t>(D.w_gate) & 31u)))
     return false;
   if (D.d_model % BK::kTileCols || D.d_model / BK::kTileCols > BK::kMaxTiles) return false;
+  if (h->nwords > BK::kMaxWords) return false;
   const int nm = D.act == PI_ACT_SWIGLU ? 2 : 1;
   if (BK::smem_bytes(D.d_model, nm) > 200 * 1024) return false;
   return (D.d_ffn + G - 1) / G <= BK::kMaxLoc;
@@ -531,10 +536,9 @@ pi_status run_ffn_batch(const pi_ffn *h, const void *u, int B, float *out, int a
   a.f = D.d_ffn;
   a.B = B;
   a.mask = w.mask();
+  a.uwords = w.uwords();
   a.nwords = h->nwords;
   a.ulist = w.ulist();
-  a.ucount = w.ucount();
-  a.uprefix = w.uprefix();
   a.hot_dense = want_dense(h, B, flags) ? 1 : 0;
   a.H = h->H;
   a.a_hi = w.b_ahi();
