@@ -58,7 +58,8 @@ constexpr int kTok = 8;          // token columns (batches of 2..8; rows past B 
 constexpr int kKStep = 64;       // elements of one step-3 unit
 constexpr int kTileCols = 64;    // columns of y per step-4 tile
 constexpr int kPosStep = 16;     // list positions per step-4 unit
-constexpr int kStages = 4;       // step-4 stages per warp
+constexpr int kStages = 3;       // step-4 stages per warp (2 units in flight; shared memory is kept
+                                 // small, since register loads need L1 room)
 constexpr int kRowBytes = kTileCols * 2;
 constexpr int kStageBytes = kPosStep * kRowBytes + 2 * kTok * kPosStep * 2;  // rows + a_hi + a_lo
 constexpr int kMaxLoc = 512;     // list positions one CTA takes in step 3
@@ -95,7 +96,7 @@ inline __host__ __device__ size_t step3_bytes(int d, int nmat) {
   return (size_t)kTok * (2 * (size_t)d + 16) + (size_t)kWarps * kMaxSlots * nmat * 128 * 4;
 }
 inline __host__ __device__ size_t step4_bytes() {
-  return (size_t)kWarps * kStages * kStageBytes + (size_t)kWarps * kPieceFloats * 4;
+  return (size_t)kWarps * kStages * kStageBytes;
 }
 inline __host__ __device__ size_t smem_bytes(int d, int nmat) {
   const size_t a = step3_bytes(d, nmat), b = step4_bytes();
@@ -108,9 +109,11 @@ PI_DEV void ldmatrix_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                : "r"(addr));
 }
-// 32 bytes (32-byte aligned) of a weight row, read once: bypass L1
+// 32 bytes (32-byte aligned) of a weight row, read once: bypass L1.
+// Volatile, so the load is issued where it is written (ahead of its use, or
+// before the grid-dependency wait) instead of being sunk to its first use.
 PI_DEV void ld_stream32(const void *p, uint4 &lo, uint4 &hi) {
-  asm("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+  asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
       : "=r"(lo.x), "=r"(lo.y), "=r"(lo.z), "=r"(lo.w), "=r"(hi.x), "=r"(hi.y), "=r"(hi.z), "=r"(hi.w)
       : "l"(p));
 }
@@ -122,15 +125,20 @@ template <int N>
 PI_DEV void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
-PI_DEV int ld_cg_i32(const int32_t *p) {
-  int v;
-  asm volatile("ld.global.cg.s32 %0, [%1];" : "=r"(v) : "l"(p));
-  return v;
-}
-// position of the k-th (0-based) set bit of w (k < popc(w))
+// position of the k-th (0-based) set bit of w (k < popc(w)): halve the
+// window by the popcount of its low half, five times
 PI_DEV int select_bit(uint32_t w, int k) {
-  for (int i = 0; i < k; ++i) w &= w - 1u;
-  return __ffs(w) - 1;
+  int pos = 0;
+#pragma unroll
+  for (int width = 16; width >= 1; width >>= 1) {
+    const int c = __popc(w & ((1u << width) - 1u));
+    if (k >= c) {
+      k -= c;
+      pos += width;
+      w >>= width;
+    }
+  }
+  return pos;
 }
 PI_DEV void st_shared_zero16(uint32_t dst) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
@@ -209,10 +217,11 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
     const int x = uidx(p);
     return x < 0 ? p : id_of_uidx(x);
   };
-  // after the grid-wide wait: the list written by the CTAs in step 3
+  // after the grid-wide wait: the list written by the CTAs in step 3 (no
+  // line of it is read by this SM before that wait, so L1 holds no stale copy)
   auto vid = [&](int p) -> int {
     const int x = uidx(p);
-    return x < 0 ? p : ld_cg_i32(a.ulist + x);
+    return x < 0 ? p : a.ulist[x];
   };
 
   // ---- step-4 spans (known once the list length is): CTA c owns units
@@ -414,7 +423,9 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
 
   // ================================================================ step 4
   const uint32_t ring = smem_u32(smem) + (uint32_t)(warp * kStages * kStageBytes);
-  float *tred = reinterpret_cast<float *>(smem + (size_t)kWarps * kStages * kStageBytes);
+  // a warp's partial of a finished tile goes to its stage that is free at
+  // that point (the one consumed last); free_s tells the others where
+  __shared__ int free_s[kWarps];
   const char *Wd = reinterpret_cast<const char *>(a.w_down_t);
   int K = 0;
   for (int t = ta; t <= tb; ++t) K += warp_count(t, warp);
@@ -493,12 +504,11 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
   for (int t = ta; t <= tb; ++t) {
     const int nt = warp_count(t, warp);
     for (int n = 0; n < nt; ++n, ++k) {
+      static_assert(kStages == 3, "the waits below count the groups of a 3-stage ring");
       if (k == 0)
         cp_async_wait<0>();
-      else if (k == 1)
-        cp_async_wait<1>();
       else
-        cp_async_wait<kStages - 2>();
+        cp_async_wait<1>();
       __syncwarp();
       const uint32_t st = ring + (uint32_t)((k % kStages) * kStageBytes);
       const uint32_t ab = st + kPosStep * kRowBytes;
@@ -520,10 +530,13 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
       issue(k + kStages - 1, ids_next, true, true);
       fetch_ids(k + kStages, ids_next, false);
     }
-    // this warp's partial of tile t
+    // this warp's partial of tile t, in its free stage (k units consumed:
+    // units k .. k + kStages - 2 are in flight, stage (k - 1) mod kStages is free)
+    const int fs = (k + kStages - 1) % kStages;
+    if (lane == 0) free_s[warp] = fs;
 #pragma unroll
     for (int mt = 0; mt < 4; ++mt) {
-      float *dst = tred + (size_t)warp * kPieceFloats;
+      float *dst = reinterpret_cast<float *>(smem + (size_t)(warp * kStages + fs) * kStageBytes);
       const int col = 16 * mt + g;
       *reinterpret_cast<float2 *>(dst + col * kTok + 2 * q) =
           make_float2(acc_h[mt][0] + acc_l[mt][0], acc_h[mt][1] + acc_l[mt][1]);
@@ -537,7 +550,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
     const int col = tid >> 3, tok = tid & 7;
     float v = 0.f;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) v += tred[(size_t)w * kPieceFloats + tid];
+    for (int w = 0; w < kWarps; ++w)
+      v += reinterpret_cast<const float *>(smem + (size_t)(w * kStages + free_s[w]) * kStageBytes)[tid];
     const long long tlo = (long long)t * S, thi = tlo + S;
     const int cf = span_owner(W, tlo, G), cl = span_owner(W, thi - 1, G);
     float *y = a.out + (size_t)tok * d + (size_t)t * kTileCols + col;
