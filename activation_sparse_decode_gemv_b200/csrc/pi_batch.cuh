@@ -609,8 +609,7 @@ struct PredArgs {
 };
 constexpr int kPredHRows = 8;   // P1 rows per CTA (MMA rows 0..7; rows 8..15 are zero)
 constexpr int kPredHUnits = 8;  // 64-element units per warp (d <= 8192)
-constexpr int kPredSWarps = 8;  // pred_s: 2 groups of 16 rows x 4 quarters of the rank
-constexpr int kPredSUnits = 4;  // units per warp (rank <= 1024)
+constexpr int kPredSUnits = 2;  // pred_s: units per warp (2 groups x 8 parts of the rank <= 1024)
 
 PI_DEV uint4 ld_cg16(const void *p) {
   uint4 v;
@@ -684,88 +683,115 @@ __global__ void __launch_bounds__(kThreads) pred_h_batch_kernel(const __grid_con
   }
 }
 
-// s_i = P2_i . h + bias_i and the fired bits for the 32 rows of CTA
-// blockIdx.x (one mask word per token).  Warp w: group w & 1 (16 rows),
-// quarter w >> 1 of the rank; B operand = h split into fp16 h_hi and
-// h_lo = fp16(h - h_hi), as two MMAs, so h enters with about 22 bits.
-__global__ void __launch_bounds__(kPredSWarps * 32) pred_s_batch_kernel(const __grid_constant__ PredArgs a) {
-  __shared__ float red[kPredSWarps][128];
+// s_i = P2_i . h + bias_i and the fired bits, 32 rows (one mask word per
+// token) at a time.  One CTA per SM walks the words c, c + G, ...; warp w
+// takes group w & 1 (16 rows) and the eighth w >> 1 of the rank, so its
+// slice of h is the same for every word: its B fragments (h split into fp16
+// h_hi and h_lo = fp16(h - h_hi), two MMAs, about 22 bits of h) are built
+// once.  The next word's rows are loaded while the current one is reduced,
+// and the first two words' rows before the grid-dependency wait.
+struct PredSBuf {
+  uint4 w[kPredSUnits][4];  // [unit][row g lo, row g hi, row g+8 lo, row g+8 hi]
+};
+__global__ void __launch_bounds__(kThreads, 1) pred_s_batch_kernel(const __grid_constant__ PredArgs a) {
+  __shared__ float red[kWarps][128];
   __shared__ uint32_t uw_s[kTok];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, q = lane & 3;
-  const int r = a.r, f = a.f;
-  const int grp = warp & 1, qr = warp >> 1;
-  const int i0 = blockIdx.x * 32 + 16 * grp + g, i1 = i0 + 8;
+  const int r = a.r, f = a.f, nw = a.nwords;
+  const int grp = warp & 1, part = warp >> 1;
   const int nsr = r / kKStep;
-  const int u0 = nsr * qr / 4, u1 = nsr * (qr + 1) / 4;
-  uint4 a0l[kPredSUnits], a0h[kPredSUnits], a1l[kPredSUnits], a1h[kPredSUnits];
+  const int u0 = nsr * part / 8, u1 = nsr * (part + 1) / 8;
+  auto load = [&](PredSBuf &b, int word) {
+    const int i0 = word * 32 + 16 * grp + g, i1 = i0 + 8;
 #pragma unroll
-  for (int i = 0; i < kPredSUnits; ++i) {
-    a0l[i] = a0h[i] = a1l[i] = a1h[i] = make_uint4(0u, 0u, 0u, 0u);
-    if (u0 + i < u1) {
-      const size_t off = (size_t)(u0 + i) * kKStep + q * 16;
-      if (i0 < f) ld_stream32(a.p2 + (size_t)i0 * r + off, a0l[i], a0h[i]);
-      if (i1 < f) ld_stream32(a.p2 + (size_t)i1 * r + off, a1l[i], a1h[i]);
+    for (int i = 0; i < kPredSUnits; ++i) {
+      b.w[i][0] = b.w[i][1] = b.w[i][2] = b.w[i][3] = make_uint4(0u, 0u, 0u, 0u);
+      if (word < nw && u0 + i < u1) {
+        const size_t off = (size_t)(u0 + i) * kKStep + q * 16;
+        if (i0 < f) ld_stream32(a.p2 + (size_t)i0 * r + off, b.w[i][0], b.w[i][1]);
+        if (i1 < f) ld_stream32(a.p2 + (size_t)i1 * r + off, b.w[i][2], b.w[i][3]);
+      }
     }
-  }
+  };
+  PredSBuf b0, b1;
+  const int G = gridDim.x;
+  int word = blockIdx.x;
+  load(b0, word);
+  load(b1, word + G);
   pdl_wait();
   pdl_launch_dependents();
-  float acc_h[4] = {0.f, 0.f, 0.f, 0.f}, acc_l[4] = {0.f, 0.f, 0.f, 0.f};
+  // this warp's h fragments: token g, unit elements 16q .. 16q + 15
+  uint32_t hh[kPredSUnits][8], hl[kPredSUnits][8];
+#pragma unroll
+  for (int i = 0; i < kPredSUnits; ++i)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      hh[i][e] = hl[i][e] = 0u;
+    }
 #pragma unroll
   for (int i = 0; i < kPredSUnits; ++i) {
-    if (u0 + i < u1) {
-      // token g's h at the unit's elements 16q .. 16q + 15, as fp16 hi / lo pairs
-      uint32_t hh[8], hl[8];
+    if (g < a.B && u0 + i < u1) {
+      const float *hp = a.h + (size_t)g * r + (size_t)(u0 + i) * kKStep + q * 16;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) hh[e] = hl[e] = 0u;
-      if (g < a.B) {
-        const float *hp = a.h + (size_t)g * r + (size_t)(u0 + i) * kKStep + q * 16;
-#pragma unroll
-        for (int v4 = 0; v4 < 4; ++v4) {
-          const float4 x = ld_cg_f4(hp + 4 * v4);
-          hh[2 * v4] = fused::h_part_pair(x.x, x.y, 0);
-          hl[2 * v4] = fused::h_part_pair(x.x, x.y, 1);
-          hh[2 * v4 + 1] = fused::h_part_pair(x.z, x.w, 0);
-          hl[2 * v4 + 1] = fused::h_part_pair(x.z, x.w, 1);
-        }
+      for (int v4 = 0; v4 < 4; ++v4) {
+        const float4 x = ld_cg_f4(hp + 4 * v4);
+        hh[i][2 * v4] = fused::h_part_pair(x.x, x.y, 0);
+        hl[i][2 * v4] = fused::h_part_pair(x.x, x.y, 1);
+        hh[i][2 * v4 + 1] = fused::h_part_pair(x.z, x.w, 0);
+        hl[i][2 * v4 + 1] = fused::h_part_pair(x.z, x.w, 1);
       }
-      const uint4 &x0 = a0l[i], &x1 = a0h[i], &y0 = a1l[i], &y1 = a1h[i];
-      const uint32_t A0[4] = {x0.x, y0.x, x0.y, y0.y}, A1[4] = {x0.z, y0.z, x0.w, y0.w};
-      const uint32_t A2[4] = {x1.x, y1.x, x1.y, y1.y}, A3[4] = {x1.z, y1.z, x1.w, y1.w};
-      mma_16816(acc_h, A0, hh[0], hh[1]);
-      mma_16816(acc_l, A0, hl[0], hl[1]);
-      mma_16816(acc_h, A1, hh[2], hh[3]);
-      mma_16816(acc_l, A1, hl[2], hl[3]);
-      mma_16816(acc_h, A2, hh[4], hh[5]);
-      mma_16816(acc_l, A2, hl[4], hl[5]);
-      mma_16816(acc_h, A3, hh[6], hh[7]);
-      mma_16816(acc_l, A3, hl[6], hl[7]);
     }
   }
+  auto word_out = [&](const PredSBuf &b, int wd) {
+    float acc_h[4] = {0.f, 0.f, 0.f, 0.f}, acc_l[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int e = 0; e < 4; ++e) red[warp][lane * 4 + e] = acc_h[e] + acc_l[e];
-  if (tid < kTok) uw_s[tid] = 0u;
-  __syncthreads();
-  // warp t: token t, lane = row of the word (group lane >> 4, M row lane & 15)
-  {
-    const int t = warp, row = lane, gr = row >> 4, m = row & 15;
-    const int ln = (m & 7) * 4 + (t >> 1), e = (t & 1) + ((m >> 3) << 1);
-    const int i = blockIdx.x * 32 + row;
-    float s = 0.f;
-#pragma unroll
-    for (int qq = 0; qq < 4; ++qq) s += red[2 * qq + gr][ln * 4 + e];
-    const bool fire = t < a.B && i < f && s + a.p_bias[i < f ? i : 0] > 0.f;
-    const uint32_t bits = __ballot_sync(0xffffffffu, fire);
-    if (lane == 0) {
-      if (t < a.B) a.mask[(size_t)t * a.nwords + blockIdx.x] = bits;
-      uw_s[t] = bits;
+    for (int i = 0; i < kPredSUnits; ++i) {
+      if (u0 + i < u1) {
+        const uint4 &x0 = b.w[i][0], &x1 = b.w[i][1], &y0 = b.w[i][2], &y1 = b.w[i][3];
+        const uint32_t A0[4] = {x0.x, y0.x, x0.y, y0.y}, A1[4] = {x0.z, y0.z, x0.w, y0.w};
+        const uint32_t A2[4] = {x1.x, y1.x, x1.y, y1.y}, A3[4] = {x1.z, y1.z, x1.w, y1.w};
+        mma_16816(acc_h, A0, hh[i][0], hh[i][1]);
+        mma_16816(acc_l, A0, hl[i][0], hl[i][1]);
+        mma_16816(acc_h, A1, hh[i][2], hh[i][3]);
+        mma_16816(acc_l, A1, hl[i][2], hl[i][3]);
+        mma_16816(acc_h, A2, hh[i][4], hh[i][5]);
+        mma_16816(acc_l, A2, hl[i][4], hl[i][5]);
+        mma_16816(acc_h, A3, hh[i][6], hh[i][7]);
+        mma_16816(acc_l, A3, hl[i][6], hl[i][7]);
+      }
     }
-  }
-  __syncthreads();
-  if (tid == 0) {
-    uint32_t u = 0u;
 #pragma unroll
-    for (int t = 0; t < kTok; ++t) u |= uw_s[t];
-    a.uwords[blockIdx.x] = u;
+    for (int e = 0; e < 4; ++e) red[warp][lane * 4 + e] = acc_h[e] + acc_l[e];
+    __syncthreads();
+    // warps 0..7: token t = warp, lane = row of the word (group lane >> 4)
+    if (warp < kTok) {
+      const int t = warp, row = lane, gr = row >> 4, m = row & 15;
+      const int ln = (m & 7) * 4 + (t >> 1), e = (t & 1) + ((m >> 3) << 1);
+      const int i = wd * 32 + row;
+      float sv = 0.f;
+#pragma unroll
+      for (int pp = 0; pp < 8; ++pp) sv += red[2 * pp + gr][ln * 4 + e];
+      const bool fire = t < a.B && i < f && sv + a.p_bias[i < f ? i : 0] > 0.f;
+      const uint32_t bits = __ballot_sync(0xffffffffu, fire);
+      if (lane == 0) {
+        if (t < a.B) a.mask[(size_t)t * nw + wd] = bits;
+        uw_s[t] = bits;
+      }
+    }
+    __syncthreads();
+    if (tid == 0) {
+      uint32_t u = 0u;
+#pragma unroll
+      for (int t = 0; t < kTok; ++t) u |= uw_s[t];
+      a.uwords[wd] = u;
+    }
+  };
+  for (; word < nw; word += 2 * G) {
+    word_out(b0, word);
+    load(b0, word + 2 * G);
+    if (word + G >= nw) break;
+    word_out(b1, word + G);
+    load(b1, word + 3 * G);
   }
 }
 

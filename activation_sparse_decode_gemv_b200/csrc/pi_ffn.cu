@@ -390,7 +390,7 @@ bool want_dense(const pi_ffn *h, int B, unsigned flags) {
 bool pred_batch_ok(const pi_ffn *h, int B) {
   const pi_ffn_desc &D = h->d;
   if (B < 2 || B > pi::batch::kTok || D.ptype != PI_W_F16) return false;
-  if (D.rank % 64 || D.rank > 64 * 4 * pi::batch::kPredSUnits) return false;
+  if (D.rank % 64 || D.rank > 64 * 8 * pi::batch::kPredSUnits) return false;
   if (D.d_model % 64 || D.d_model > 64 * pi::batch::kWarps * pi::batch::kPredHUnits) return false;
   return !((reinterpret_cast<uintptr_t>(D.p1) | reinterpret_cast<uintptr_t>(D.p2)) & 31u);
 }
@@ -418,7 +418,8 @@ pi_status run_predict(const pi_ffn *h, const void *u, int B, int32_t *idx, int i
     a.nwords = h->nwords;
     PI_CUDA(launch(pi::batch::pred_h_batch_kernel, dim3(cdiv(D.rank, pi::batch::kPredHRows)),
                    dim3(pi::batch::kThreads), st, a));
-    PI_CUDA(launch(pi::batch::pred_s_batch_kernel, dim3(h->nwords), dim3(pi::batch::kPredSWarps * 32), st, a));
+    PI_CUDA(launch(pi::batch::pred_s_batch_kernel, dim3(h->nwords < w.L.G ? h->nwords : w.L.G),
+                   dim3(pi::batch::kThreads), st, a));
     if (idx || count || !batch_ok(h, B, w.L.G))
       PI_CUDA(launch(pi::compact_kernel, dim3(B + 1), dim3(1024), st, (const uint32_t *)w.mask(), h->nwords,
                      idx_stride, B, idx, count, w.uwords(), w.uprefix(), w.ulist(), w.ucount()));
