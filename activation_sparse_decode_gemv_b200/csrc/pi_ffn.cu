@@ -222,7 +222,11 @@ bool build_fused_map(pi_ffn *h) {
   return h->fx_ok;
 }
 
-constexpr int kTcMinBatch = 16;
+// Smallest batch that takes the tensor-core path: int4 layers from 2 tokens
+// (the CUDA-core batch kernel reads fp16 rows only), fp16 layers from 9 (the
+// CUDA-core batch kernel covers 2..8).
+int tc_min_batch(const pi_ffn *h) { return h->d.wtype == PI_W_INT4G32 ? 2 : 9; }
+bool tc_ok(const pi_ffn *h, int B);
 
 struct Ws {
   WsLayout L;
@@ -272,7 +276,9 @@ pi_status get_ws(const pi_ffn *const *layers, int n, int B, void *ws, size_t ws_
   out->L = ws_layout(dmax, fmax, rmax, B, G);
   out->base = static_cast<char *>(ws);
   out->tc = nullptr;
-  if (B >= kTcMinBatch) {
+  bool tc = false;
+  for (int i = 0; i < n; ++i) tc = tc || tc_ok(layers[i], B);
+  if (tc) {
     out->T = tc_layout(dmax, fmax, rmax, G);
     if (out->T.total > ws_bytes) return PI_ERR_WORKSPACE;
     const uintptr_t end = reinterpret_cast<uintptr_t>(ws) + ws_bytes;
@@ -610,9 +616,10 @@ pi_status run_ffn(const pi_ffn *h, const void *u, int B, float *out, int accumul
 namespace TC = pi::tc;
 
 // The tcgen05 kernels take fp16 predictors and fp16 or int4 weights (int4
-// rows in whole 256-element scale blocks; see build_tc_maps) at 16 <= B <= 32.
+// rows in whole 256-element scale blocks; see build_tc_maps) at
+// tc_min_batch <= B <= 32 (token columns past B are zero).
 bool tc_ok(const pi_ffn *h, int B) {
-  return B >= kTcMinBatch && B <= TC::kN && h->tc_maps && h->d.d_ffn <= TC::kMaxTiles * TC::kM;
+  return B >= tc_min_batch(h) && B <= TC::kN && h->tc_maps && h->d.d_ffn <= TC::kMaxTiles * TC::kM;
 }
 
 template <typename KArg>
@@ -981,7 +988,9 @@ pi_status pi_workspace_size(const pi_ffn_t *layers, int n_layers, int max_batch,
   const int G = device_sm_count();
   if (G <= 0) return PI_ERR_CUDA;
   *bytes = ws_layout(dmax, fmax, rmax, max_batch, G).total;
-  if (max_batch >= kTcMinBatch) *bytes += tc_layout(dmax, fmax, rmax, G).total + 256;
+  bool tc = false;
+  for (int i = 0; i < n_layers; ++i) tc = tc || (layers[i]->tc_maps && max_batch >= tc_min_batch(layers[i]));
+  if (tc) *bytes += tc_layout(dmax, fmax, rmax, G).total + 256;
   return PI_OK;
 }
 

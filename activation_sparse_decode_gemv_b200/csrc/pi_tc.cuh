@@ -753,7 +753,11 @@ __global__ void __launch_bounds__(RowShape<KIND, WT, ACT>::THREADS, 1) row_gemm_
         }
         if (lane == 0 && any) atomicOr(a.uwords + word, any);  // union words (order-free)
       } else {
-        // a image position: listed tile j_tile, row m
+        // a image position: listed tile j_tile, row m.  Up to 16 tokens the
+        // image holds a_hi = fp16(a) in column n and a_lo = fp16(a - a_hi) in
+        // column n + 16 (the down GEMM adds the two), so a keeps about 22
+        // bits; above 16 tokens every column is a token and a is fp16(a).
+        const bool split = a.B <= kN / 2;
         const bool valid = row < a.nrows;
         const float b1 = (ACT == ACT_RELU && valid) ? __ldg(a.bias + row) : 0.f;
         const long long pos = j_tile * kM + m;
@@ -761,6 +765,7 @@ __global__ void __launch_bounds__(RowShape<KIND, WT, ACT>::THREADS, 1) row_gemm_
 #pragma unroll
         for (int j = 0; j < S::TOKW; ++j) {
           const int n = kq * S::TOKW + j;
+          if (split && n >= kN / 2) continue;  // column of a lo part, written below
           float av = 0.f;
           if (valid && n < a.B) {
             const uint32_t bits = __ldg(a.mask + (size_t)n * a.nwords + (row >> 5));
@@ -773,7 +778,11 @@ __global__ void __launch_bounds__(RowShape<KIND, WT, ACT>::THREADS, 1) row_gemm_
               }
             }
           }
-          *reinterpret_cast<__half *>(a.out0 + boff + img_off(n, (int)(pos & 15))) = __float2half_rn(av);
+          const __half hi = __float2half_rn(av);
+          *reinterpret_cast<__half *>(a.out0 + boff + img_off(n, (int)(pos & 15))) = hi;
+          if (split)
+            *reinterpret_cast<__half *>(a.out0 + boff + img_off(n + kN / 2, (int)(pos & 15))) =
+                __float2half_rn(av - __half2float(hi));
         }
       }
     }
@@ -998,12 +1007,14 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_down_kernel(const __grid_cons
                                          abort_flag, a.status, &ok))
         continue;
       const int dpos = (int)tile * kDownTileD + hm * kM + q * 32 + lane;
+      const bool split = a.B <= kN / 2;  // columns n + 16 hold the a_lo parts
       if (dpos < d) {
 #pragma unroll
         for (int n = 0; n < kN; ++n) {
           if (n < a.B) {
+            const float yv = split ? v[n] + v[(n + kN / 2) % kN] : v[n];
             float *yp = a.y + (size_t)n * d + dpos;
-            *yp = a.accumulate ? *yp + v[n] : v[n];
+            *yp = a.accumulate ? *yp + yv : yv;
           }
         }
       }
