@@ -39,16 +39,23 @@ import torch
 from activation_sparse_decode_gemv_b200 import inputs
 
 def kernels_per_step(cfg, B, ids=False):
-    """Launches of the library's kernels per decode step: batch 1 with fp16 /
-    int4 weights runs as one persistent fused kernel; batches 16..32 with fp16
-    / int4 weights run five (token image, two tensor-core predictor GEMMs,
-    tensor-core up/gate and down GEMMs), plus the compaction when the call
-    asks for the id lists (``ids``); otherwise five kernels (predictor stage
-    1, stage 2, compaction, gather, reduction)."""
+    """Launches of the library's kernels per decode step (the library's
+    dispatch, see pi_decode_ffn in include/pi_ffn.h): batch 1 with fp16 / int4
+    weights runs as one persistent fused kernel; int4 batches of 2..32 and
+    fp16 batches of 9..32 run five on the tensor-core path (token image, two
+    predictor GEMMs, up/gate and down GEMMs); fp16 batches of 2..8 run three
+    (two predictor kernels, the persistent FFN kernel); the compaction adds
+    one when the call asks for the id lists (``ids``); anything else runs five
+    CUDA-core kernels (predictor stage 1, stage 2, compaction, gather,
+    reduction)."""
     if B == 1 and cfg.wtype != "f32" and cfg.r <= 1024 and cfg.d <= 8192:
         return 1
-    if 16 <= B <= 32 and cfg.wtype != "f32" and (cfg.wtype != "int4g32" or cfg.d % 256 == 0):
+    tc_min = 2 if cfg.wtype == "int4g32" else 9
+    if tc_min <= B <= 32 and cfg.wtype != "f32" and (cfg.wtype != "int4g32" or cfg.d % 256 == 0):
         return 6 if ids else 5
+    if (2 <= B <= 8 and cfg.wtype == "f16" and cfg.d % 64 == 0 and cfg.d <= 8192 and cfg.r % 64 == 0
+            and cfg.r <= 1024 and cfg.f <= 32768):
+        return 4 if ids else 3
     return 5
 
 
@@ -72,6 +79,10 @@ def parse(argv=None):
     ap.add_argument("--stack-config", default="opt30b_stack_f16",
                     help="stacked workload timed as the line's 'stack' object at batch 1 ('none' skips it)")
     ap.add_argument("--stack-steps", type=int, default=200)
+    ap.add_argument("--batch-configs", default="opt7b_f16:8,llama13b_swiglu_f16:4,llama70b_swiglu_int4:4,"
+                    "llama70b_swiglu_int4:32",
+                    help="config:batch pairs timed as the line's 'batches' objects ('none' skips them)")
+    ap.add_argument("--batch-steps", type=int, default=400)
     ap.add_argument("--json-out", default=None)
     ap.add_argument("--stack", action="store_true",
                     help="time pi_decode_ffn_stack through all layers of a stacked config (tokens/s)")
@@ -535,6 +546,8 @@ def bench_ours(args, world, rank, local):
     }
     if args.stack_config != "none":
         line["stack"] = stack_summary(args, world, rank, local)
+    if args.batch_configs != "none":
+        line["batches"] = [batch_summary(args, world, rank, local, spec) for spec in args.batch_configs.split(",")]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         host = layers[0].to("cpu")
         del layers, handles
@@ -584,6 +597,24 @@ def stack_summary(args, world, rank, local):
             "bytes_per_token": st["config"]["bytes_per_step"], "roofline": st["roofline"],
             "gpu_launches_per_token": st["gpu_launches_per_step"], "clocks": st["clocks"],
             "generation_s": st["config"]["generation_s"]}
+
+
+def batch_summary(args, world, rank, local, spec):
+    """One multi-token single-layer configuration (``config:batch``), timed
+    like the main line (rotating replicas larger than L2, CUDA graphs, CUDA
+    events), for the line's 'batches' objects."""
+    import copy
+    name, b = spec.split(":")
+    a = copy.copy(args)
+    a.config, a.batch, a.replicas, a.tokens = name, int(b), 4, 8
+    a.steps, a.warmup, a.e2e_steps = args.batch_steps, max(3, args.batch_steps // 10), 16
+    a.stack_config, a.batch_configs, a.no_cpu_baseline, a.cpu_workers, a.rank = "none", "none", True, 0, 0
+    ln = bench_ours(a, world, rank, local)
+    torch.cuda.empty_cache()
+    return {"workload": ln["config"]["workload"], "batch": a.batch, "us_per_layer": ln["us_per_layer"],
+            "value": ln["value"], "unit": ln["unit"], "steps": ln["steps"], "warmup": ln["warmup"],
+            "bytes_per_step": ln["config"]["bytes_per_step"], "roofline": ln["roofline"],
+            "gpu_launches_per_step": ln["gpu_launches"] // ln["steps"], "clocks": ln["clocks"]}
 
 
 def bench_stack(args, world, rank, local):
