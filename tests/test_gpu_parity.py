@@ -216,3 +216,34 @@ def test_repeated_decode_is_bitwise_stable(cuda_device, name, B):
     bad = sum(int(not torch.equal(g.decode(u)[0], y0)) for _ in range(200))
     assert bad == 0, f"{bad} of 200 repeated decodes differ"
     assert g.status() == 0
+
+
+# ------------------------------------------------------------------ every batch size of each path
+
+@pytest.mark.parametrize("name,batches", [
+    ("opt7b_f16", list(range(2, 17))),             # batch kernels 2..8, tcgen05 9..16
+    ("llama13b_swiglu_f16", [2, 5, 7, 8, 9, 12]),
+    ("llama70b_swiglu_int4", [2, 3, 5, 6]),        # tcgen05 from 2 tokens (int4)
+])
+def test_every_batch_size_matches_the_oracle(cuda_device, name, batches):
+    """Predictor, sparse FFN and decode step against the oracle at each batch
+    size, across the boundaries where the library changes kernels (the fp16
+    batch kernels end at 8 tokens, the tensor-core path starts at 9 for fp16
+    and at 2 for int4)."""
+    cfg = small_cfg(name, d=1024 if name != "llama70b_swiglu_int4" else 512)
+    lt = inputs.make_layer(cfg, 0, seed=83)
+    g = Gpu(lt, 16)
+    for B in batches:
+        u = inputs.layer_input(cfg, inputs.make_tokens(cfg, B, B, seed=89))
+        check_layer(lt, u, g)
+
+
+def test_batch_on_a_width_the_batch_kernels_do_not_take(cuda_device):
+    """d = 520 is not a multiple of 64: batches 2..8 run on the CUDA-core
+    multi-kernel path, which must match the oracle as well."""
+    cfg = small_cfg("opt7b_f16", d=520)
+    lt = inputs.make_layer(cfg, 0, seed=97)
+    g = Gpu(lt, 8)
+    for B in (2, 5, 8):
+        u = inputs.layer_input(cfg, inputs.make_tokens(cfg, B, B, seed=101))
+        check_layer(lt, u, g)
