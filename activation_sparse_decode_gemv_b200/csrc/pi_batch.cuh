@@ -19,10 +19,11 @@
 // lines per instruction were measured to cost HBM more than half its
 // bandwidth).  Those are A fragments once the K order inside the unit is
 // permuted the same way for the token operand (a dot product does not depend
-// on the order of its terms).  The tokens sit in shared memory.  The CTA's units are split into 16 contiguous spans, one per
-// warp (stream-K inside the CTA); each warp leaves one partial per group it
-// touched in shared memory and the CTA adds them in warp order.  The
-// activation a (zero for tokens that did not predict the neuron) is stored as
+// on the order of its terms).  The tokens sit in shared memory.  Warp w
+// takes the units w, w + 16, ... of every group, so the 16 warps read one
+// contiguous 2 KB run of each of the group's rows together; each leaves its
+// partial of the group in shared memory (double-buffered by group) and, after
+// the group's barrier, the CTA adds them in warp order.  The activation a (zero for tokens that did not predict the neuron) is stored as
 // two fp16 parts, a_hi = fp16(a) and a_lo = fp16(a - a_hi), so step 4 carries
 // a to about 22 bits.
 //
@@ -63,7 +64,6 @@ constexpr int kStages = 3;       // step-4 stages per warp (2 units in flight; s
 constexpr int kRowBytes = kTileCols * 2;
 constexpr int kStageBytes = kPosStep * kRowBytes + 2 * kTok * kPosStep * 2;  // rows + a_hi + a_lo
 constexpr int kMaxLoc = 512;     // list positions one CTA takes in step 3
-constexpr int kMaxSlots = 3;     // groups one warp's step-3 span touches (kMaxLoc / 16 <= 32 groups)
 constexpr int kMaxTiles = 192;   // step-4 tiles (d <= 12288)
 constexpr int kMaxWords = 1024;  // 32-neuron words of the union (d_ffn <= 32768)
 constexpr int kPieceFloats = kTileCols * kTok;
@@ -93,7 +93,7 @@ struct Args {
 // dynamic shared memory: step 3 (tokens + warp partials) and step 4 (stages +
 // tile partials) use the same bytes, one after the other
 inline __host__ __device__ size_t step3_bytes(int d, int nmat) {
-  return (size_t)kTok * (2 * (size_t)d + 16) + (size_t)kWarps * kMaxSlots * nmat * 128 * 4;
+  return (size_t)kTok * (2 * (size_t)d + 16) + (size_t)2 * kWarps * nmat * 128 * 4;
 }
 inline __host__ __device__ size_t step4_bytes() {
   return (size_t)kWarps * kStages * kStageBytes;
@@ -162,7 +162,6 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
   __shared__ uint32_t memb_s[kMaxLoc];
   __shared__ float bias_s[kMaxLoc];
   __shared__ int last_s;
-  __shared__ int span_lo_s[kWarps], span_jlo_s[kWarps], span_jhi_s[kWarps];
   __shared__ uint32_t uw_s[kMaxWords];
   __shared__ int pre_s[kMaxWords + 1];  // exclusive prefix of the union words' popcounts
   __shared__ int wsum_s[kWarps];
@@ -298,21 +297,16 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
 
   const int ns = d / kKStep;
   const int ng = (nloc + 15) >> 4;
-  const int T = ng * ns;
-  const int w0 = T * warp / kWarps, w1 = T * (warp + 1) / kWarps;
-  const int ja = w0 / ns;
-  if (tid < kWarps) {  // each warp's span, for the reduction (T * 16 < 2^31)
-    const int lo = T * tid / kWarps, hi = T * (tid + 1) / kWarps;
-    span_lo_s[tid] = lo < hi ? 1 : 0;
-    span_jlo_s[tid] = lo / ns;
-    span_jhi_s[tid] = lo < hi ? (hi - 1) / ns : -1;
-  }
+  // warp w takes the steps w, w + 16, ... of every group, so the 16 warps
+  // read one contiguous 2 KB run of each of the group's rows at a time
+  const int per = ns > warp ? (ns - warp + kWarps - 1) / kWarps : 0;
+  const int nu = ng * per;  // this warp's units
   {
     struct Buf {
       uint4 w[NM][4];  // [matrix][row g elements 0-7, 8-15, row g+8 elements 0-7, 8-15] of this lane's 16
     };
     auto load = [&](Buf &bf, int ui) {
-      const int j = ui / ns, s = ui - j * ns;
+      const int j = ui / per, s = warp + kWarps * (ui - j * per);
       const int r0 = 16 * j + g, r1 = r0 + 8;
       const size_t off = (size_t)s * (kKStep * 2) + (size_t)q * 32;
 #pragma unroll
@@ -333,8 +327,46 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
     for (int m = 0; m < NM; ++m)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[m][e] = 0.f;
+    // group j's partials: red[j % 2][warp][matrix][lane * 4 + e]
+    auto flush = [&](int j) {
+#pragma unroll
+      for (int m = 0; m < NM; ++m) {
+        float *dst = red + ((size_t)(((j & 1) * kWarps + warp) * NM + m) * 128) + lane * 4;
+        *reinterpret_cast<float4 *>(dst) = make_float4(acc[m][0], acc[m][1], acc[m][2], acc[m][3]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[m][e] = 0.f;
+      }
+    };
+    // after group j's barrier: the sums over the warps in warp order,
+    // activation, membership; a by list position
+    auto reduce_group = [&](int j) {
+      if (tid < 128) {
+        const int rm = tid >> 3, t = tid & 7, p = 16 * j + rm;
+        if (p < nloc) {
+          const int ln = (rm & 7) * 4 + (t >> 1), e = (t & 1) + ((rm >> 3) << 1);
+          float x[NM];
+#pragma unroll
+          for (int m = 0; m < NM; ++m) x[m] = 0.f;
+#pragma unroll 4
+          for (int w = 0; w < kWarps; ++w)
+#pragma unroll
+            for (int m = 0; m < NM; ++m) x[m] += red[(size_t)(((j & 1) * kWarps + w) * NM + m) * 128 + ln * 4 + e];
+          float av = 0.f;
+          if ((memb_s[p] >> t) & 1u) {
+            if constexpr (ACT == ACT_RELU)
+              av = fmaxf(x[0] + bias_s[p], 0.f);
+            else
+              av = silu(x[1]) * x[0];
+          }
+          const __half hi = __float2half_rn(av);
+          const __half lo = __float2half_rn(av - __half2float(hi));
+          a.a_hi[(size_t)t * a.a_stride + pb + p] = hi;
+          a.a_lo[(size_t)t * a.a_stride + pb + p] = lo;
+        }
+      }
+    };
     auto compute = [&](const Buf &bf, int ui) {
-      const int j = ui / ns, s = ui - j * ns;
+      const int j = ui / per, i = ui - j * per, s = warp + kWarps * i;
       // token g's elements 16q .. 16q + 15 of the unit, the same K order as the rows
       const __half *ur = u_s + (size_t)g * upitch + (size_t)s * kKStep + q * 16;
       const uint4 ub0 = *reinterpret_cast<const uint4 *>(ur), ub1 = *reinterpret_cast<const uint4 *>(ur + 8);
@@ -358,58 +390,35 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
           mma_16816(acc[m], A, ub1.z, ub1.w);
         }
       }
-      if (s == ns - 1 || ui == w1 - 1) {  // end of this warp's part of group j
-#pragma unroll
-        for (int m = 0; m < NM; ++m) {
-          float *dst = red + ((size_t)((warp * kMaxSlots + (j - ja)) * NM + m) * 128) + lane * 4;
-          *reinterpret_cast<float4 *>(dst) = make_float4(acc[m][0], acc[m][1], acc[m][2], acc[m][3]);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) acc[m][e] = 0.f;
-        }
+      if (i == per - 1) {  // this warp's last step of group j
+        flush(j);
+        __syncthreads();
+        reduce_group(j);
       }
     };
-    Buf buf[PD];
+    if (per == 0) {  // a warp with no step (d < 1024): zeros, and the same barriers
+      for (int j = 0; j < ng; ++j) {
+        flush(j);
+        __syncthreads();
+        reduce_group(j);
+      }
+    } else {
+      // loads run PD - 1 units ahead of the MMAs, across group ends
+      Buf buf[PD];
 #pragma unroll
-    for (int k = 0; k < PD - 1; ++k)
-      if (w0 + k < w1) load(buf[k], w0 + k);
-    for (int ui = w0; ui < w1; ui += PD) {
+      for (int k = 0; k < PD - 1; ++k)
+        if (k < nu) load(buf[k], k);
+      for (int ui = 0; ui < nu; ui += PD) {
 #pragma unroll
-      for (int k = 0; k < PD; ++k) {
-        const int uk = ui + k;
-        if (uk < w1) {
-          if (uk + PD - 1 < w1) load(buf[(k + PD - 1) % PD], uk + PD - 1);
-          compute(buf[k], uk);
+        for (int k = 0; k < PD; ++k) {
+          const int uk = ui + k;
+          if (uk < nu) {
+            if (uk + PD - 1 < nu) load(buf[(k + PD - 1) % PD], uk + PD - 1);
+            compute(buf[k], uk);
+          }
         }
       }
     }
-  }
-  __syncthreads();
-  // sums over the warps in warp order, activation, membership; a by position
-  for (int it = tid; it < ng * 128; it += kThreads) {
-    const int j = it >> 7, rm = (it >> 3) & 15, t = it & 7;
-    const int p = 16 * j + rm;
-    if (p >= nloc) continue;
-    const int ln = (rm & 7) * 4 + (t >> 1), e = (t & 1) + ((rm >> 3) << 1);
-    float x[NM];
-#pragma unroll
-    for (int m = 0; m < NM; ++m) x[m] = 0.f;
-    for (int w = 0; w < kWarps; ++w) {
-      const int jlo = span_jlo_s[w];
-      if (!span_lo_s[w] || j < jlo || j > span_jhi_s[w]) continue;
-#pragma unroll
-      for (int m = 0; m < NM; ++m) x[m] += red[(size_t)((w * kMaxSlots + (j - jlo)) * NM + m) * 128 + ln * 4 + e];
-    }
-    float av = 0.f;
-    if ((memb_s[p] >> t) & 1u) {
-      if constexpr (ACT == ACT_RELU)
-        av = fmaxf(x[0] + bias_s[p], 0.f);
-      else
-        av = silu(x[1]) * x[0];
-    }
-    const __half hi = __float2half_rn(av);
-    const __half lo = __float2half_rn(av - __half2float(hi));
-    a.a_hi[(size_t)t * a.a_stride + pb + p] = hi;
-    a.a_lo[(size_t)t * a.a_stride + pb + p] = lo;
   }
   // the positions past the list up to the next multiple of 16 read as zero
   if (c == G - 1 && tid < kTok * kPosStep) {
