@@ -438,45 +438,69 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
   const char *Wd = reinterpret_cast<const char *>(a.w_down_t);
   int K = 0;
   for (int t = ta; t <= tb; ++t) K += warp_count(t, warp);
-  auto unit_of = [&](int k, int &t, int &s) { unit_of_w(k, warp, t, s); };
-  auto issue_acts = [&](int k) {
-    int t, s;
-    unit_of(k, t, s);
+  // walks this warp's units in order (k-th unit = (tile t, step s)); one step
+  // costs a few integer operations, so the per-unit bookkeeping stays off the
+  // path of the copies
+  struct Cursor {
+    int k, t, s, rem;  // rem: this warp's units of tile t after this one
+  };
+  auto cursor_tile = [&](Cursor &cu) {  // first unit of the first tile >= cu.t with units
+    for (; cu.t <= tb; ++cu.t) {
+      const int n = warp_count(cu.t, warp);
+      if (n > 0) {
+        int sa, sb;
+        tile_steps(cu.t, sa, sb);
+        cu.s = sa + warp;
+        cu.rem = n - 1;
+        return;
+      }
+    }
+  };
+  auto cursor_next = [&](Cursor &cu) {
+    ++cu.k;
+    if (cu.rem > 0) {
+      cu.s += kWarps;
+      --cu.rem;
+    } else {
+      ++cu.t;
+      cursor_tile(cu);
+    }
+  };
+  Cursor fc{0, ta, 0, 0};
+  cursor_tile(fc);
+  auto issue_acts = [&](int k, int s) {
     const uint32_t st = ring + (uint32_t)((k % kStages) * kStageBytes);
     const int hl = lane >> 4, t8 = (lane >> 1) & 7, half = lane & 1;
     const __half *src = (hl ? a.a_lo : a.a_hi) + (size_t)t8 * a.a_stride + (size_t)s * kPosStep + half * 8;
     cp_async16(st + (uint32_t)(kPosStep * kRowBytes + hl * (kTok * kPosStep * 2) + t8 * 32 + half * 16), src);
   };
-  // list ids of the rows this lane copies for unit k (rows lane / 8 + 4 i),
-  // fetched one unit ahead so the copies do not wait for them
-  auto fetch_ids = [&](int k, int (&id)[4], bool local) {
-    if (k < K) {
-      int t, s;
-      unit_of(k, t, s);
+  // list ids of the rows this lane copies for the cursor's unit (rows
+  // lane / 8 + 4 i), fetched one unit ahead of its copies
+  auto fetch_ids = [&](const Cursor &cu, int (&id)[4], bool local) {
+    if (cu.k < K) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const int row = (lane >> 3) + 4 * i, p = s * kPosStep + row;
-        id[i] = local ? pro_ids_s[warp][k][row] : (p < V ? vid(p) : -1);
+        const int row = (lane >> 3) + 4 * i, p = cu.s * kPosStep + row;
+        id[i] = local ? pro_ids_s[warp][cu.k][row] : (p < V ? vid(p) : -1);
       }
     }
   };
-  auto issue = [&](int k, const int (&id)[4], bool rows, bool acts) {
+  auto issue = [&](int k, int t, int s, const int (&id)[4], bool rows, bool acts) {
     if (k < K) {
-      int t, s;
-      unit_of(k, t, s);
       const uint32_t st = ring + (uint32_t)((k % kStages) * kStageBytes);
       if (rows) {
+        const char *col = Wd + (size_t)t * kRowBytes + (lane & 7) * 16;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int row = (lane >> 3) + 4 * i, ch = lane & 7;
           const uint32_t dst = st + (uint32_t)(row * kRowBytes + ((ch ^ (row & 7)) << 4));
           if (id[i] >= 0)
-            cp_async16(dst, Wd + (size_t)id[i] * rb + (size_t)t * kRowBytes + ch * 16);
+            cp_async16(dst, col + (size_t)id[i] * rb);
           else
             st_shared_zero16(dst);
         }
       }
-      if (acts) issue_acts(k);
+      if (acts) issue_acts(k, s);
     }
     cp_async_commit();
   };
@@ -484,18 +508,24 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
   // the first stages' weight rows do not depend on step 3: in flight during
   // the grid-wide wait
   int ids_next[4];
+  int pro_s[kStages - 1];
 #pragma unroll
   for (int k = 0; k < kStages - 1; ++k) {
-    fetch_ids(k, ids_next, true);
-    issue(k, ids_next, true, false);
+    fetch_ids(fc, ids_next, true);
+    issue(k, fc.t, fc.s, ids_next, true, false);
+    pro_s[k] = fc.s;
+    cursor_next(fc);
   }
-  fetch_ids(kStages - 1, ids_next, true);
+  fetch_ids(fc, ids_next, true);
+  int nx_t = fc.t, nx_s = fc.s;  // the unit ids_next belong to (unit kStages - 1)
+  cursor_next(fc);
   if (tid == 0) grid_barrier(a.bar, G, c, a.status, a.wait_ns);
   __syncthreads();
   pdl_launch_dependents();
   // their activations, as one more group
+#pragma unroll
   for (int k = 0; k < kStages - 1; ++k)
-    if (k < K) issue_acts(k);
+    if (k < K) issue_acts(k, pro_s[k]);
   cp_async_commit();
 
   if (W == 0) {  // empty list: y = 0
@@ -536,8 +566,11 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
         mma_16816(acc_l[mt], A, bl0, bl1);
       }
       __syncwarp();
-      issue(k + kStages - 1, ids_next, true, true);
-      fetch_ids(k + kStages, ids_next, false);
+      issue(k + kStages - 1, nx_t, nx_s, ids_next, true, true);
+      fetch_ids(fc, ids_next, false);
+      nx_t = fc.t;
+      nx_s = fc.s;
+      cursor_next(fc);
     }
     // this warp's partial of tile t, in its free stage (k units consumed:
     // units k .. k + kStages - 2 are in flight, stage (k - 1) mod kStages is free)
