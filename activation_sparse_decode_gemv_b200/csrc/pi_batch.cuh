@@ -305,22 +305,35 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
     struct Buf {
       uint4 w[NM][4];  // [matrix][row g elements 0-7, 8-15, row g+8 elements 0-7, 8-15] of this lane's 16
     };
-    auto load = [&](Buf &bf, int ui) {
-      const int j = ui / per, s = warp + kWarps * (ui - j * per);
-      const int r0 = 16 * j + g, r1 = r0 + 8;
-      const size_t off = (size_t)s * (kKStep * 2) + (size_t)q * 32;
+    // load cursor: group lj, step index li; the group's row pointers are
+    // looked up once per group (integer work per unit stays small)
+    int lj = -1, li = per;
+    const char *rp0[NM], *rp1[NM];
+    auto load = [&](Buf &bf) {
+      if (li == per) {
+        li = 0;
+        ++lj;
+        const int r0 = 16 * lj + g, r1 = r0 + 8;
+#pragma unroll
+        for (int m = 0; m < NM; ++m) {
+          const char *W = reinterpret_cast<const char *>(m == 0 ? a.w_up : a.w_gate);
+          rp0[m] = r0 < nloc ? W + (size_t)ids_s[r0] * rb + (size_t)q * 32 : nullptr;
+          rp1[m] = r1 < nloc ? W + (size_t)ids_s[r1] * rb + (size_t)q * 32 : nullptr;
+        }
+      }
+      const size_t off = (size_t)(warp + kWarps * li) * (kKStep * 2);
 #pragma unroll
       for (int m = 0; m < NM; ++m) {
-        const char *W = reinterpret_cast<const char *>(m == 0 ? a.w_up : a.w_gate);
-        if (r0 < nloc)
-          ld_stream32(W + (size_t)ids_s[r0] * rb + off, bf.w[m][0], bf.w[m][1]);
+        if (rp0[m])
+          ld_stream32(rp0[m] + off, bf.w[m][0], bf.w[m][1]);
         else
           bf.w[m][0] = bf.w[m][1] = make_uint4(0u, 0u, 0u, 0u);
-        if (r1 < nloc)
-          ld_stream32(W + (size_t)ids_s[r1] * rb + off, bf.w[m][2], bf.w[m][3]);
+        if (rp1[m])
+          ld_stream32(rp1[m] + off, bf.w[m][2], bf.w[m][3]);
         else
           bf.w[m][2] = bf.w[m][3] = make_uint4(0u, 0u, 0u, 0u);
       }
+      ++li;
     };
     float acc[NM][4];
 #pragma unroll
@@ -365,8 +378,13 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
         }
       }
     };
-    auto compute = [&](const Buf &bf, int ui) {
-      const int j = ui / per, i = ui - j * per, s = warp + kWarps * i;
+    int cj = 0, ci = 0;  // compute cursor: group, step index
+    auto compute = [&](const Buf &bf) {
+      const int j = cj, i = ci, s = warp + kWarps * i;
+      if (++ci == per) {
+        ci = 0;
+        ++cj;
+      }
       // token g's elements 16q .. 16q + 15 of the unit, the same K order as the rows
       const __half *ur = u_s + (size_t)g * upitch + (size_t)s * kKStep + q * 16;
       const uint4 ub0 = *reinterpret_cast<const uint4 *>(ur), ub1 = *reinterpret_cast<const uint4 *>(ur + 8);
@@ -407,14 +425,14 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
       Buf buf[PD];
 #pragma unroll
       for (int k = 0; k < PD - 1; ++k)
-        if (k < nu) load(buf[k], k);
+        if (k < nu) load(buf[k]);
       for (int ui = 0; ui < nu; ui += PD) {
 #pragma unroll
         for (int k = 0; k < PD; ++k) {
           const int uk = ui + k;
           if (uk < nu) {
-            if (uk + PD - 1 < nu) load(buf[(k + PD - 1) % PD], uk + PD - 1);
-            compute(buf[k], uk);
+            if (uk + PD - 1 < nu) load(buf[(k + PD - 1) % PD]);
+            compute(buf[k]);
           }
         }
       }
