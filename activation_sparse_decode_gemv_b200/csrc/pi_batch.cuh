@@ -651,12 +651,21 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
 
 
 // ================================================================ predictor (batches of 2..8)
-// The same tensor-core row dot as step 3: weight rows as A fragments loaded
-// with 256-bit loads (elements 16q .. 16q + 15 of a 64-element unit per
-// lane), the tokens (or h) as the B operand in the matching K order.  The
-// weight rows do not depend on the previous kernel, so each kernel loads its
-// rows into registers before griddepcontrol.wait: P2 streams in while P1 is
-// still being reduced.
+// One persistent kernel, one CTA per SM, for steps 1-2 of a token batch.  It
+// uses the same tensor-core row dot as step 3: weight rows as A fragments
+// loaded with 256-bit loads (elements 16q .. 16q + 15 of a 64-element unit
+// per lane), the tokens (or h) as the B operand in the matching K order.
+//   P1: CTA c computes h for P1 rows 8c .. 8c + 7 (MMA rows 8..15 are zero),
+//       K = d split over the 16 warps, partials added in warp order.
+//   one grid-wide wait (bounded): h complete.
+//   P2: the CTA walks the 32-row words c, c + G, ... (one mask word per
+//       token); warp w takes group w & 1 (16 rows) and the eighth w >> 1 of
+//       the rank, so its B fragments of h (split into fp16 h_hi and
+//       h_lo = fp16(h - h_hi), two MMAs, about 22 bits of h) are built once.
+//       The next word's rows are loaded while the current one is reduced.
+// Neither P1 nor P2 rows depend on the previous kernel: the CTA's P1 rows and
+// its first P2 word are loaded before griddepcontrol.wait, and the first
+// word is in registers while P1 is reduced and h exchanged.
 struct PredArgs {
   const __half *p1, *p2;
   const float *p_bias;
@@ -666,10 +675,13 @@ struct PredArgs {
   uint32_t *mask;    // [B x nwords]
   uint32_t *uwords;  // [nwords], OR of the tokens' words
   int nwords;
+  unsigned *bar;     // grid-barrier word
+  int *status;
+  unsigned long long wait_ns;
 };
-constexpr int kPredHRows = 8;   // P1 rows per CTA (MMA rows 0..7; rows 8..15 are zero)
-constexpr int kPredHUnits = 8;  // 64-element units per warp (d <= 8192)
-constexpr int kPredSUnits = 2;  // pred_s: units per warp (2 groups x 8 parts of the rank <= 1024)
+constexpr int kPredHRows = 8;   // P1 rows per CTA
+constexpr int kPredHUnits = 8;  // P1 64-element units per warp (d <= 8192)
+constexpr int kPredSUnits = 2;  // P2 units per warp (2 groups x 8 parts of the rank <= 1024)
 
 PI_DEV uint4 ld_cg16(const void *p) {
   uint4 v;
@@ -682,14 +694,18 @@ PI_DEV float4 ld_cg_f4(const float *p) {
   return v;
 }
 
-// h[t][j] = P1_j . u_t for the 8 rows j of CTA blockIdx.x; warp w takes the
-// units [w ns / 16, (w + 1) ns / 16) of the d / 64 units, the CTA adds the
-// warps' partials in warp order.
-__global__ void __launch_bounds__(kThreads) pred_h_batch_kernel(const __grid_constant__ PredArgs a) {
-  __shared__ float red[kWarps][64];
+struct PredSBuf {
+  uint4 w[kPredSUnits][4];  // [unit][row g lo, row g hi, row g+8 lo, row g+8 hi]
+};
+__global__ void __launch_bounds__(kThreads, 1) pred_batch_kernel(const __grid_constant__ PredArgs a) {
+  __shared__ float red[kWarps][128];
+  __shared__ uint32_t uw_s[kTok];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, q = lane & 3;
-  const int d = a.d, r = a.r;
-  const int j = blockIdx.x * kPredHRows + g;
+  const int G = gridDim.x, c = blockIdx.x;
+  const int d = a.d, r = a.r, f = a.f, nw = a.nwords;
+
+  // ---- P1 rows of this CTA, and its first P2 word, before the wait
+  const int j = c * kPredHRows + g;
   const int ns = d / kKStep;
   const int w0 = ns * warp / kWarps, w1 = ns * (warp + 1) / kWarps;
   uint4 wl[kPredHUnits], wh[kPredHUnits];
@@ -698,66 +714,6 @@ __global__ void __launch_bounds__(kThreads) pred_h_batch_kernel(const __grid_con
     wl[i] = wh[i] = make_uint4(0u, 0u, 0u, 0u);
     if (w0 + i < w1 && j < r) ld_stream32(a.p1 + (size_t)j * d + (size_t)(w0 + i) * kKStep + q * 16, wl[i], wh[i]);
   }
-  pdl_wait();
-  pdl_launch_dependents();
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-  for (int i = 0; i < kPredHUnits; ++i) {
-    if (w0 + i < w1) {
-      uint4 ub0 = make_uint4(0u, 0u, 0u, 0u), ub1 = ub0;
-      if (g < a.B) {
-        const __half *up = a.u + (size_t)g * d + (size_t)(w0 + i) * kKStep + q * 16;
-        ub0 = ld_cg16(up);
-        ub1 = ld_cg16(up + 8);
-      }
-      const uint4 &x0 = wl[i], &x1 = wh[i];
-      {
-        const uint32_t A[4] = {x0.x, 0u, x0.y, 0u};
-        mma_16816(acc, A, ub0.x, ub0.y);
-      }
-      {
-        const uint32_t A[4] = {x0.z, 0u, x0.w, 0u};
-        mma_16816(acc, A, ub0.z, ub0.w);
-      }
-      {
-        const uint32_t A[4] = {x1.x, 0u, x1.y, 0u};
-        mma_16816(acc, A, ub1.x, ub1.y);
-      }
-      {
-        const uint32_t A[4] = {x1.z, 0u, x1.w, 0u};
-        mma_16816(acc, A, ub1.z, ub1.w);
-      }
-    }
-  }
-  // lane (g, q) holds row g, tokens 2q and 2q + 1
-  red[warp][lane * 2] = acc[0];
-  red[warp][lane * 2 + 1] = acc[1];
-  __syncthreads();
-  if (tid < kPredHRows * kTok) {
-    const int row = tid >> 3, t = tid & 7;
-    const int jr = blockIdx.x * kPredHRows + row;
-    float v = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) v += red[w][(row * 4 + (t >> 1)) * 2 + (t & 1)];
-    if (t < a.B && jr < r) a.h[(size_t)t * r + jr] = v;
-  }
-}
-
-// s_i = P2_i . h + bias_i and the fired bits, 32 rows (one mask word per
-// token) at a time.  One CTA per SM walks the words c, c + G, ...; warp w
-// takes group w & 1 (16 rows) and the eighth w >> 1 of the rank, so its
-// slice of h is the same for every word: its B fragments (h split into fp16
-// h_hi and h_lo = fp16(h - h_hi), two MMAs, about 22 bits of h) are built
-// once.  The next word's rows are loaded while the current one is reduced,
-// and the first two words' rows before the grid-dependency wait.
-struct PredSBuf {
-  uint4 w[kPredSUnits][4];  // [unit][row g lo, row g hi, row g+8 lo, row g+8 hi]
-};
-__global__ void __launch_bounds__(kThreads, 1) pred_s_batch_kernel(const __grid_constant__ PredArgs a) {
-  __shared__ float red[kWarps][128];
-  __shared__ uint32_t uw_s[kTok];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, q = lane & 3;
-  const int r = a.r, f = a.f, nw = a.nwords;
   const int grp = warp & 1, part = warp >> 1;
   const int nsr = r / kKStep;
   const int u0 = nsr * part / 8, u1 = nsr * (part + 1) / 8;
@@ -774,13 +730,62 @@ __global__ void __launch_bounds__(kThreads, 1) pred_s_batch_kernel(const __grid_
     }
   };
   PredSBuf b0, b1;
-  const int G = gridDim.x;
-  int word = blockIdx.x;
+  int word = c;
   load(b0, word);
-  load(b1, word + G);
   pdl_wait();
+
+  // ---- P1: h[t][j] = P1_j . u_t
+  {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < kPredHUnits; ++i) {
+      if (w0 + i < w1) {
+        uint4 ub0 = make_uint4(0u, 0u, 0u, 0u), ub1 = ub0;
+        if (g < a.B) {
+          const __half *up = a.u + (size_t)g * d + (size_t)(w0 + i) * kKStep + q * 16;
+          ub0 = ld_cg16(up);
+          ub1 = ld_cg16(up + 8);
+        }
+        const uint4 &x0 = wl[i], &x1 = wh[i];
+        {
+          const uint32_t A[4] = {x0.x, 0u, x0.y, 0u};
+          mma_16816(acc, A, ub0.x, ub0.y);
+        }
+        {
+          const uint32_t A[4] = {x0.z, 0u, x0.w, 0u};
+          mma_16816(acc, A, ub0.z, ub0.w);
+        }
+        {
+          const uint32_t A[4] = {x1.x, 0u, x1.y, 0u};
+          mma_16816(acc, A, ub1.x, ub1.y);
+        }
+        {
+          const uint32_t A[4] = {x1.z, 0u, x1.w, 0u};
+          mma_16816(acc, A, ub1.z, ub1.w);
+        }
+      }
+    }
+    // lane (g, q) holds row g, tokens 2q and 2q + 1
+    red[warp][lane * 2] = acc[0];
+    red[warp][lane * 2 + 1] = acc[1];
+    __syncthreads();
+    if (tid < kPredHRows * kTok) {
+      const int row = tid >> 3, t = tid & 7;
+      const int jr = c * kPredHRows + row;
+      float v = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) v += red[w][(row * 4 + (t >> 1)) * 2 + (t & 1)];
+      if (t < a.B && jr < r) a.h[(size_t)t * r + jr] = v;
+    }
+    __syncthreads();
+  }
+  // every CTA's slice of h written
+  if (tid == 0) grid_barrier(a.bar, G, c, a.status, a.wait_ns);
+  __syncthreads();
   pdl_launch_dependents();
-  // this warp's h fragments: token g, unit elements 16q .. 16q + 15
+  load(b1, word + G);
+
+  // ---- P2: this warp's h fragments, token g, unit elements 16q .. 16q + 15
   uint32_t hh[kPredSUnits][8], hl[kPredSUnits][8];
 #pragma unroll
   for (int i = 0; i < kPredSUnits; ++i)

@@ -390,6 +390,15 @@ bool want_dense(const pi_ffn *h, int B, unsigned flags) {
     if ((call) != cudaSuccess) return PI_ERR_CUDA; \
   } while (0)
 
+// Test support (pi_debug_wait_fault): an entry of h that is never published,
+// and a shorter limit for every bounded wait of the fused and batch
+// kernels.
+struct WaitFault {
+  int withhold = -1;
+  unsigned long long limit_ns = 0;  // 0: the kernel's default
+};
+WaitFault g_wait_fault;
+
 // The tensor-core predictor kernels of batches 2..8: fp16 predictor, rank a
 // multiple of 64 up to 1024, d a multiple of 64 up to 8192, P1 and P2 on
 // 32-byte boundaries (256-bit row loads).
@@ -398,6 +407,8 @@ bool pred_batch_ok(const pi_ffn *h, int B) {
   if (B < 2 || B > pi::batch::kTok || D.ptype != PI_W_F16) return false;
   if (D.rank % 64 || D.rank > 64 * 8 * pi::batch::kPredSUnits) return false;
   if (D.d_model % 64 || D.d_model > 64 * pi::batch::kWarps * pi::batch::kPredHUnits) return false;
+  // one CTA per SM computes 8 rows of h
+  if (D.rank > pi::batch::kPredHRows * device_sm_count()) return false;
   return !((reinterpret_cast<uintptr_t>(D.p1) | reinterpret_cast<uintptr_t>(D.p2)) & 31u);
 }
 
@@ -422,10 +433,10 @@ pi_status run_predict(const pi_ffn *h, const void *u, int B, int32_t *idx, int i
     a.mask = w.mask();
     a.uwords = w.uwords();
     a.nwords = h->nwords;
-    PI_CUDA(launch(pi::batch::pred_h_batch_kernel, dim3(cdiv(D.rank, pi::batch::kPredHRows)),
-                   dim3(pi::batch::kThreads), st, a));
-    PI_CUDA(launch(pi::batch::pred_s_batch_kernel, dim3(h->nwords < w.L.G ? h->nwords : w.L.G),
-                   dim3(pi::batch::kThreads), st, a));
+    a.bar = w.grid_bar();
+    a.status = w.status();
+    a.wait_ns = g_wait_fault.limit_ns ? g_wait_fault.limit_ns : pi::batch::kWaitNs;
+    PI_CUDA(launch(pi::batch::pred_batch_kernel, dim3(w.L.G), dim3(pi::batch::kThreads), st, a));
     if (idx || count || !batch_ok(h, B, w.L.G))
       PI_CUDA(launch(pi::compact_kernel, dim3(B + 1), dim3(1024), st, (const uint32_t *)w.mask(), h->nwords,
                      idx_stride, B, idx, count, w.uwords(), w.uprefix(), w.ulist(), w.ucount()));
@@ -478,14 +489,6 @@ pi_status run_sets(const pi_ffn *h, const int32_t *idx, const int32_t *count, in
   return PI_OK;
 }
 
-// Test support (pi_debug_wait_fault): an entry of h that is never published,
-// and a shorter limit for every bounded wait of the fused and batch
-// kernels.
-struct WaitFault {
-  int withhold = -1;
-  unsigned long long limit_ns = 0;  // 0: the kernel's default
-};
-WaitFault g_wait_fault;
 
 // ---------------------------------------------------------------- batch kernel (2..8 tokens)
 namespace BK = pi::batch;
