@@ -664,8 +664,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
 //       h_lo = fp16(h - h_hi), two MMAs, about 22 bits of h) are built once.
 //       The next word's rows are loaded while the current one is reduced.
 // Neither P1 nor P2 rows depend on the previous kernel: the CTA's P1 rows and
-// its first P2 word are loaded before griddepcontrol.wait, and the first
-// word is in registers while P1 is reduced and h exchanged.
+// its first P2 word are loaded before griddepcontrol.wait, the second word
+// before the grid-wide wait, so both are in flight while h is exchanged.
 struct PredArgs {
   const __half *p1, *p2;
   const float *p_bias;
@@ -779,11 +779,12 @@ __global__ void __launch_bounds__(kThreads, 1) pred_batch_kernel(const __grid_co
     }
     __syncthreads();
   }
+  // the second word's rows stream in during the wait (the P1 registers are free)
+  load(b1, word + G);
   // every CTA's slice of h written
   if (tid == 0) grid_barrier(a.bar, G, c, a.status, a.wait_ns);
   __syncthreads();
   pdl_launch_dependents();
-  load(b1, word + G);
 
   // ---- P2: this warp's h fragments, token g, unit elements 16q .. 16q + 15
   uint32_t hh[kPredSUnits][8], hl[kPredSUnits][8];

@@ -48,12 +48,12 @@ def test_launch_claims_match_the_launch_lists():
     # profiles/launch_list_opt7b_f16_batch1.md: one decode_fused_kernel per step
     assert bench.kernels_per_step(C["opt7b_f16"], 1) == 1
     assert bench.kernels_per_step(C["llama70b_swiglu_int4"], 1) == 1
-    # profiles/launch_list_llama13b_f16_batch4.md: pred_h, pred_s, the FFN kernel
+    # profiles/launch_list_llama13b_f16_batch4.md: the predictor kernel, the FFN kernel
     # (the compaction only when the step asks for the id lists)
-    assert bench.kernels_per_step(C["llama13b_swiglu_f16"], 4) == 3
-    assert bench.kernels_per_step(C["llama13b_swiglu_f16"], 4, ids=True) == 4
-    # profiles/launch_list_opt7b_f16_batch8.md: the same three at batch 8
-    assert bench.kernels_per_step(C["opt7b_f16"], 8) == 3
+    assert bench.kernels_per_step(C["llama13b_swiglu_f16"], 4) == 2
+    assert bench.kernels_per_step(C["llama13b_swiglu_f16"], 4, ids=True) == 3
+    # profiles/launch_list_opt7b_f16_batch8.md: the same two at batch 8
+    assert bench.kernels_per_step(C["opt7b_f16"], 8) == 2
     # profiles/launch_list_llama70b_int4_batch4.md: int4 from 2 tokens on the tensor-core path
     assert bench.kernels_per_step(C["llama70b_swiglu_int4"], 4) == 5
     # profiles/launch_list_llama70b_int4_batch32.md: u_image, P1, P2, up/gate, down
@@ -68,8 +68,8 @@ def test_launch_list_summaries_have_the_claimed_kernels():
     def kernel_rows(name):
         with open(os.path.join(ROOT, "profiles", name)) as fh:
             return [l for l in fh if l.startswith("| `")]
-    assert len(kernel_rows("launch_list_llama13b_f16_batch4.md")) == 3
-    assert len(kernel_rows("launch_list_opt7b_f16_batch8.md")) == 3
+    assert len(kernel_rows("launch_list_llama13b_f16_batch4.md")) == 2
+    assert len(kernel_rows("launch_list_opt7b_f16_batch8.md")) == 2
     assert len(kernel_rows("launch_list_llama70b_int4_batch4.md")) == 5
     assert len(kernel_rows("launch_list_llama70b_int4_batch32.md")) == 5
 
