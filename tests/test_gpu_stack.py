@@ -131,3 +131,43 @@ def test_full_stack(cuda_device, name):
         assert_outputs(xo.cpu().numpy().astype(np.float64) - xl.numpy().astype(np.float64), y_ref, cfg.wtype,
                        f"layer {l}")
         del lt, L
+
+
+@pytest.mark.slow
+def test_full_stack_batch4():
+    """The 40-layer LLaMA-13B-shaped stack at its listed batch of 4 (the
+    batch kernels, accumulating into x): one decode step through every layer,
+    then the first and last layer as one-layer stacks against the oracle on
+    seeded 4-token inputs (sets outside the rounding band identical, each
+    token's update within the fp16 tolerance)."""
+    cfg = inputs.CONFIGS["llama13b_swiglu_f16"]
+    B = 4
+    dev = torch.device("cuda")
+    layers = [inputs.make_layer(cfg, l, seed=0, device=dev) for l in range(cfg.n_layers)]
+    handles = [pb.FfnLayer.from_tensors(l) for l in layers]
+    ws = pb.make_workspace(handles, B, dev)
+    x = inputs.make_tokens(cfg, 0, B, seed=0).to(dev)
+    idx = torch.empty((cfg.n_layers, B, cfg.f), dtype=torch.int32, device=dev)
+    cnt = torch.empty((cfg.n_layers, B), dtype=torch.int32, device=dev)
+    xs = x.clone()
+    pb.pi_decode_ffn_stack(handles, xs, ws, idx_trace=idx, count_trace=cnt)
+    assert pb.pi_get_device_status(ws) == 0
+    c = cnt.cpu().numpy()
+    assert abs(c.mean() / cfg.f - cfg.mean_p) < 0.35 * cfg.mean_p, c.mean() / cfg.f
+    assert torch.isfinite(xs).all()
+    for l in (0, cfg.n_layers - 1):
+        lt = layers[l].to("cpu")
+        L = host_layer(lt)
+        xl = inputs.make_tokens(cfg, 100 + l, B, seed=0)
+        u, _ = oracle.rmsnorm_f16(xl.numpy())
+        pr = oracle.predict(L, u)
+        xo = xl.to(dev)
+        ii = torch.empty((1, B, cfg.f), dtype=torch.int32, device=dev)
+        cc = torch.empty((1, B), dtype=torch.int32, device=dev)
+        pb.pi_decode_ffn_stack([handles[l]], xo, ws, idx_trace=ii, count_trace=cc)
+        got = [ii.cpu().numpy()[0, b, :int(cc[0, b].item())] for b in range(B)]
+        sets, flips, _ = compare_sets(got, pr, cfg.f)
+        y_ref = oracle.ffn_masked(L, u, sets)
+        assert_outputs(xo.cpu().numpy().astype(np.float64) - xl.numpy().astype(np.float64), y_ref, cfg.wtype,
+                       f"layer {l}")
+        del lt, L
