@@ -172,6 +172,22 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
   const size_t rb = (size_t)d * 2;
 
   pdl_wait();
+  // the tokens into shared memory (rows B..7 zero), in flight during the
+  // union scan; cp.async, so the copy needs no registers
+  const int upitch = d + 8;  // halves; rows 16 bytes apart modulo 128 (conflict-free fragment reads)
+  __half *u_s = reinterpret_cast<__half *>(smem);
+  {
+    const int dch = d / 8;
+    for (int k = tid; k < kTok * dch; k += kThreads) {
+      const int t = k / dch, e = k - t * dch;
+      const uint32_t dst = smem_u32(u_s + (size_t)t * upitch + (size_t)e * 8);
+      if (t < B)
+        cp_async16(dst, a.u + (size_t)t * d + (size_t)e * 8);
+      else
+        st_shared_zero16(dst);
+    }
+    cp_async_commit();
+  }
   // ---- the union: every CTA scans the union words itself (same result in
   // every CTA), so no separate compaction runs before this kernel
   const int nw = a.nwords;
@@ -271,17 +287,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
   // ================================================================ step 3
   const int pb = list_begin(c, V, G), pe = list_begin(c + 1, V, G);
   const int nloc = pe - pb;
-  const int upitch = d + 8;  // halves; rows 16 bytes apart modulo 128 (conflict-free fragment reads)
-  __half *u_s = reinterpret_cast<__half *>(smem);
   float *red = reinterpret_cast<float *>(smem + (size_t)kTok * upitch * 2);
   {
-    const int dch = d / 8;
-    for (int k = tid; k < kTok * dch; k += kThreads) {
-      const int t = k / dch, e = k - t * dch;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (t < B) v = *reinterpret_cast<const uint4 *>(a.u + (size_t)t * d + (size_t)e * 8);
-      *reinterpret_cast<uint4 *>(u_s + (size_t)t * upitch + (size_t)e * 8) = v;
-    }
     for (int k = tid; k < nloc; k += kThreads) {
       const int x = uidx(pb + k);
       const int i = x < 0 ? pb + k : id_of_uidx(x);
@@ -293,6 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_batch_kernel(const __grid_con
       if (ACT == ACT_RELU) bias_s[k] = a.b_up[i];
     }
   }
+  cp_async_wait<0>();  // the tokens
   __syncthreads();
 
   const int ns = d / kKStep;
