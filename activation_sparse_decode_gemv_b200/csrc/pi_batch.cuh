@@ -1,17 +1,24 @@
-// pi_batch.cuh -- the FFN of a token batch of 2..8 over the union of the
-// tokens' predicted sets, as one persistent kernel per layer (PowerInfer
-// summary page: Summary, neuron-aware sparse operators; Interesting ideas I4,
-// kernels that read only the rows of the active neurons).
+// pi_batch.cuh -- the decode step of a token batch of 2..8 with fp16 weights
+// (PowerInfer summary page: Summary, per-layer predictor and neuron-aware
+// sparse operators; Interesting ideas I4, kernels that read only the rows of
+// the active neurons), as two persistent kernels per layer:
+// pred_batch_kernel (steps 1-2, at the end of this file) and
+// ffn_batch_kernel (steps 2-4 over the union of the tokens' sets).
 //
-// Grid: one CTA per SM (all co-resident; the one grid-wide wait is bounded).
-// The union list (hot prefix first in dense mode) is the K of step 3 and the
-// reduction axis of step 4.  Both steps are small matrix products with the
-// batch as N = 8 columns, so they run on the tensor cores (mma.sync
-// m16n8k16, fp16 inputs, fp32 accumulation); the work is bound by HBM, and the
-// tensor cores only keep the instruction count per weight byte low.
+// Grid: one CTA per SM (all co-resident; each kernel's one grid-wide wait is
+// bounded).  The products are small matrix products with the batch as N = 8
+// columns, so they run on the tensor cores (mma.sync m16n8k16, fp16 inputs,
+// fp32 accumulation); the work is bound by HBM, and the tensor cores only
+// keep the instruction count per weight byte low.
+//
+// ffn_batch_kernel:
+// Union.  Every CTA scans the union words (the OR of the tokens' mask
+// words) itself: block prefix of their popcounts, so a list position maps to
+// its neuron id by a binary search and a bit select.  The list is the hot
+// prefix densely (dense mode), then the union's other neurons ascending.
 //
 // Step 3 (up / gate + activation).  CTA c takes the list positions
-// [chunk_begin(c), chunk_begin(c + 1)), in groups of 16 neurons (the MMA's M).
+// [list_begin(c), list_begin(c + 1)), in groups of 16 neurons (the MMA's M).
 // A unit is 64 elements of the 16 rows of a group.  The weight rows go from
 // HBM straight into registers: lane (g, q) of a warp loads the 32 bytes at
 // elements 16q .. 16q + 15 of rows g and g + 8 (one 256-bit load each, so the
@@ -19,25 +26,31 @@
 // lines per instruction were measured to cost HBM more than half its
 // bandwidth).  Those are A fragments once the K order inside the unit is
 // permuted the same way for the token operand (a dot product does not depend
-// on the order of its terms).  The tokens sit in shared memory.  Warp w
-// takes the units w, w + 16, ... of every group, so the 16 warps read one
+// on the order of its terms).  The tokens sit in shared memory.  Warp w takes
+// the units w, w + 16, ... of every group, so the 16 warps read one
 // contiguous 2 KB run of each of the group's rows together; each leaves its
 // partial of the group in shared memory (double-buffered by group) and, after
-// the group's barrier, the CTA adds them in warp order.  The activation a (zero for tokens that did not predict the neuron) is stored as
-// two fp16 parts, a_hi = fp16(a) and a_lo = fp16(a - a_hi), so step 4 carries
-// a to about 22 bits.
+// the group's barrier, the CTA adds them in warp order.  The activation a
+// (zero for tokens that did not predict the neuron) is stored as two fp16
+// parts, a_hi = fp16(a) and a_lo = fp16(a - a_hi), so step 4 carries a to
+// about 22 bits.  The CTA also writes its positions' ids into the union list.
 //
 // Step 4 (down).  y^T [d x 8] = W2T^T [d x list] * a [list x 8].  A unit is a
 // tile of 64 columns of y times 16 list positions; units are ordered tile by
 // tile and split into G contiguous spans (stream-K over CTAs), so every CTA
-// does the same amount of work and reads 128-byte row segments.  Inside a CTA
-// the warps take the units of a tile in turn and each keeps its own ring of 4
+// does the same amount of work.  Inside a CTA the warps take the units of a
+// tile in turn (an incremental cursor walks them: per-unit bookkeeping was
+// measured to bound this stream before) and each keeps its own ring of 3
 // shared-memory stages filled with cp.async (16-byte copies, XOR-swizzled so
 // that ldmatrix.trans reads them without bank conflicts); the activations of
 // the unit's positions ride in the same stage.  A tile covered by one CTA is
 // written to y directly; a tile split between CTAs is finished by the last
-// CTA to arrive (per-tile counter), which adds the pieces in CTA order, so the
-// result does not depend on timing.  Counters reset themselves.
+// CTA to arrive (per-tile counter), which adds the pieces in CTA order, so
+// the result does not depend on timing.  Counters reset themselves.
+//
+// Shared memory stays near 150 KB: register loads need L1 room (a streaming
+// read was measured to drop from 6.3 to 4.5 TB/s with 200 KB of shared
+// memory per SM).
 #pragma once
 
 #include <cuda.h>
@@ -144,7 +157,7 @@ PI_DEV void st_shared_zero16(uint32_t dst) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
 }
 
-// range of list positions of CTA c (the same formula as the CUDA-core gather
+// first list position of CTA c (the same split as the CUDA-core gather
 // kernel)
 PI_DEV int list_begin(int c, int V, int G) { return (int)(((long long)c * V) / G); }
 
