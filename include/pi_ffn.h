@@ -39,7 +39,10 @@
  *    read back with pi_get_device_status; kernels never trap.
  *  - Alignment: every pointer 16-byte aligned; d % 8 == 0 for fp16 weights,
  *    d % 32 == 0 for int4g32, d % 4 == 0 for fp32, rank % 8 == 0 (fp16
- *    predictor) or % 4 (fp32); d <= 16384, 1 <= batch <= 32.
+ *    predictor) or % 4 (fp32); d <= 16384, 1 <= batch <= 32.  Some kernels
+ *    need more (32-byte aligned matrices, d a multiple of 64 or 256); a call
+ *    whose arguments do not meet them runs on a slower kernel that computes
+ *    the same result, never fails for it (see pi_decode_ffn).
  */
 #ifndef PI_FFN_H
 #define PI_FFN_H
@@ -117,7 +120,9 @@ void pi_ffn_destroy(pi_ffn_t h);
 pi_status pi_workspace_size(const pi_ffn_t *layers, int n_layers, int max_batch, size_t *bytes);
 
 /* Zero a workspace (cudaMemsetAsync on the stream).  Required once before
- * first use; kernels leave it reusable afterwards. */
+ * first use; kernels leave it reusable afterwards (their counters and
+ * barrier words return to their initial state at the end of every call, and
+ * a workspace may serve calls of any batch up to the size it was sized for). */
 pi_status pi_workspace_init(void *ws, size_t ws_bytes, pi_stream_t stream);
 
 /* Predictor only (steps 1-2: the per-layer predictor of the summary page's
