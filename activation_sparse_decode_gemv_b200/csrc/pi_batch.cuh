@@ -61,7 +61,6 @@
 namespace pi {
 namespace batch {
 
-using fused::globaltimer;
 using fused::grid_barrier;
 using fused::mma_16816;
 using fused::smem_u32;
