@@ -413,6 +413,7 @@ bool pred_batch_ok(const pi_ffn *h, int B) {
 }
 
 bool batch_ok(const pi_ffn *h, int B, int G);
+bool tc_ok(const pi_ffn *h, int B);
 
 // steps 1-2: predictor, mask words, compaction (idx/count optional; the batch
 // FFN kernel scans the union words itself, so without lists it needs none)
@@ -437,7 +438,10 @@ pi_status run_predict(const pi_ffn *h, const void *u, int B, int32_t *idx, int i
     a.status = w.status();
     a.wait_ns = g_wait_fault.limit_ns ? g_wait_fault.limit_ns : pi::batch::kWaitNs;
     PI_CUDA(launch(pi::batch::pred_batch_kernel, dim3(w.L.G), dim3(pi::batch::kThreads), st, a));
-    if (idx || count || !batch_ok(h, B, w.L.G))
+    // the batch FFN kernel scans the union words itself and the tensor-core
+    // FFN kernels list their tiles from them: only the multi-kernel gather
+    // needs the compacted list
+    if (idx || count || !(batch_ok(h, B, w.L.G) || tc_ok(h, B)))
       PI_CUDA(launch(pi::compact_kernel, dim3(B + 1), dim3(1024), st, (const uint32_t *)w.mask(), h->nwords,
                      idx_stride, B, idx, count, w.uwords(), w.uprefix(), w.ulist(), w.ucount()));
     return PI_OK;
@@ -1013,7 +1017,8 @@ pi_status pi_predict(pi_ffn_t h, const void *u, int B, int32_t *idx, int32_t *co
   Ws w;
   const pi_ffn *L[1] = {h};
   if ((s = get_ws(L, 1, B, ws, ws_bytes, &w)) != PI_OK) return s;
-  if (tc_ok(h, B)) return run_predict_tc(h, u, B, idx, h->d.d_ffn, count, w, (cudaStream_t)stream);
+  if (tc_ok(h, B) && !pred_batch_ok(h, B))
+    return run_predict_tc(h, u, B, idx, h->d.d_ffn, count, w, (cudaStream_t)stream);
   return run_predict(h, u, B, idx, h->d.d_ffn, count, w, (cudaStream_t)stream);
 }
 
@@ -1050,6 +1055,13 @@ pi_status pi_decode_ffn(pi_ffn_t h, const void *u, int B, float *y, int32_t *idx
   const int acc = (flags & PI_FFN_ACCUMULATE) ? 1 : 0;
   if (fused_ok(h, B, w.L.G)) return run_fused(h, u, y, 0, acc, idx, count, flags, w, st);
   if (tc_ok(h, B)) {
+    // up to 8 tokens the batch predictor (fp16 predictor whatever the
+    // weights) is the faster steps 1-2; it writes the mask and union words
+    // the tensor-core FFN kernels read
+    if (pred_batch_ok(h, B)) {
+      if ((s = run_predict(h, u, B, idx, h->d.d_ffn, count, w, st)) != PI_OK) return s;
+      return run_ffn_tc(h, u, B, y, acc, false, w, st);
+    }
     if ((s = run_predict_tc(h, u, B, idx, h->d.d_ffn, count, w, st)) != PI_OK) return s;
     return run_ffn_tc(h, u, B, y, acc, true, w, st);
   }
@@ -1086,8 +1098,13 @@ pi_status pi_decode_ffn_stack(const pi_ffn_t *layers, int L, float *x, int B, in
     }
     PI_CUDA(launch(pi::rmsnorm_kernel, dim3(B), dim3(256), st, (const float *)x, d, w.u()));
     if (tc_ok(layers[l], B)) {
-      if ((s = run_predict_tc(layers[l], w.u(), B, idx, fmax, cnt, w, st)) != PI_OK) return s;
-      if ((s = run_ffn_tc(layers[l], w.u(), B, x, 1, true, w, st)) != PI_OK) return s;
+      if (pred_batch_ok(layers[l], B)) {
+        if ((s = run_predict(layers[l], w.u(), B, idx, fmax, cnt, w, st)) != PI_OK) return s;
+        if ((s = run_ffn_tc(layers[l], w.u(), B, x, 1, false, w, st)) != PI_OK) return s;
+      } else {
+        if ((s = run_predict_tc(layers[l], w.u(), B, idx, fmax, cnt, w, st)) != PI_OK) return s;
+        if ((s = run_ffn_tc(layers[l], w.u(), B, x, 1, true, w, st)) != PI_OK) return s;
+      }
       continue;
     }
     if ((s = run_predict(layers[l], w.u(), B, idx, fmax, cnt, w, st)) != PI_OK) return s;

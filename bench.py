@@ -41,21 +41,24 @@ from activation_sparse_decode_gemv_b200 import inputs
 def kernels_per_step(cfg, B, ids=False):
     """Launches of the library's kernels per decode step (the library's
     dispatch, see pi_decode_ffn in include/pi_ffn.h): batch 1 with fp16 / int4
-    weights runs as one persistent fused kernel; int4 batches of 2..32 and
-    fp16 batches of 9..32 run five on the tensor-core path (token image, two
-    predictor GEMMs, up/gate and down GEMMs); fp16 batches of 2..8 run two
-    (the persistent predictor kernel, the persistent FFN kernel); the
-    compaction adds one when the call asks for the id lists (``ids``);
-    anything else runs five
+    weights runs as one persistent fused kernel; fp16 batches of 2..8 run two
+    (the persistent predictor kernel, the persistent FFN kernel); int4
+    batches of 2..8 run four (that predictor kernel, then the tensor-core
+    token image, up/gate and down GEMMs); int4 batches of 9..32 and fp16
+    batches of 9..32 run five on the tensor-core path (token image, two
+    predictor GEMMs, up/gate and down GEMMs); the compaction adds one when
+    the call asks for the id lists (``ids``); anything else runs five
     CUDA-core kernels (predictor stage 1, stage 2, compaction, gather,
     reduction)."""
     if B == 1 and cfg.wtype != "f32" and cfg.r <= 1024 and cfg.d <= 8192:
         return 1
+    pred_batch = (2 <= B <= 8 and cfg.wtype != "f32" and cfg.r % 64 == 0 and cfg.r <= 1024
+                  and cfg.d % 64 == 0 and cfg.d <= 8192 and cfg.r <= 8 * 148)
     tc_min = 2 if cfg.wtype == "int4g32" else 9
     if tc_min <= B <= 32 and cfg.wtype != "f32" and (cfg.wtype != "int4g32" or cfg.d % 256 == 0):
-        return 6 if ids else 5
-    if (2 <= B <= 8 and cfg.wtype == "f16" and cfg.d % 64 == 0 and cfg.d <= 8192 and cfg.r % 64 == 0
-            and cfg.r <= 1024 and cfg.f <= 32768 and cfg.r <= 8 * 148):
+        n = 4 if pred_batch else 5
+        return n + 1 if ids else n
+    if pred_batch and cfg.wtype == "f16" and cfg.f <= 32768:
         return 3 if ids else 2
     return 5
 

@@ -151,11 +151,13 @@ pi_status pi_sparse_ffn(pi_ffn_t h, const void *u, int B, const int32_t *idx, co
  *  - batch 1, fp16/int4 weights (d <= 8192): one persistent fused kernel;
  *  - batch 2..8, fp16 weights and predictor (d % 64 == 0, rank a multiple
  *    of 64 up to 1024, weight and predictor matrices 32-byte aligned):
- *    tensor-core (mma.sync) predictor kernels and one persistent FFN kernel
+ *    tensor-core (mma.sync) predictor kernel and one persistent FFN kernel
  *    over the union of the tokens' sets;
  *  - batch 9..32 with fp16 weights, or 2..32 with int4 weights (fp16
  *    predictor; int4: d % 256 == 0): tcgen05 GEMMs over the 128-neuron tiles
- *    that hold a predicted neuron of some token;
+ *    that hold a predicted neuron of some token; for int4 batches of 2..8
+ *    that meet the predictor conditions above, the batch predictor kernel
+ *    replaces the two predictor GEMMs;
  *  - otherwise: CUDA-core predictor, compaction, gather and reduction kernels.
  * Results agree within the stated tolerances whichever path runs. */
 pi_status pi_decode_ffn(pi_ffn_t h, const void *u, int B, float *y, int32_t *idx, int32_t *count, unsigned flags,

@@ -54,8 +54,10 @@ def test_launch_claims_match_the_launch_lists():
     assert bench.kernels_per_step(C["llama13b_swiglu_f16"], 4, ids=True) == 3
     # profiles/launch_list_opt7b_f16_batch8.md: the same two at batch 8
     assert bench.kernels_per_step(C["opt7b_f16"], 8) == 2
-    # profiles/launch_list_llama70b_int4_batch4.md: int4 from 2 tokens on the tensor-core path
-    assert bench.kernels_per_step(C["llama70b_swiglu_int4"], 4) == 5
+    # profiles/launch_list_llama70b_int4_batch4.md: int4 from 2 tokens on the tensor-core
+    # FFN kernels, up to 8 tokens behind the batch predictor kernel
+    assert bench.kernels_per_step(C["llama70b_swiglu_int4"], 4) == 4
+    assert bench.kernels_per_step(C["llama70b_swiglu_int4"], 4, ids=True) == 5
     # profiles/launch_list_llama70b_int4_batch32.md: u_image, P1, P2, up/gate, down
     # (no compaction when the step asks for no id lists)
     assert bench.kernels_per_step(C["llama70b_swiglu_int4"], 32) == 5
@@ -70,7 +72,7 @@ def test_launch_list_summaries_have_the_claimed_kernels():
             return [l for l in fh if l.startswith("| `")]
     assert len(kernel_rows("launch_list_llama13b_f16_batch4.md")) == 2
     assert len(kernel_rows("launch_list_opt7b_f16_batch8.md")) == 2
-    assert len(kernel_rows("launch_list_llama70b_int4_batch4.md")) == 5
+    assert len(kernel_rows("launch_list_llama70b_int4_batch4.md")) == 4
     assert len(kernel_rows("launch_list_llama70b_int4_batch32.md")) == 5
 
 
