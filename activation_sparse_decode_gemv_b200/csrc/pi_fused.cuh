@@ -23,10 +23,10 @@
 //   DONE        end of the stream
 // The producer "harvests" a tile when its slot's empty barrier completes
 // (every consumer warp is done with it), appends the fired ids to its list
-// and issues their gather rows; it keeps issuing P2 tiles meanwhile.  At the
-// start it also asks L2 for all of this CTA's P2 rows (bulk L2 prefetch), so
-// HBM keeps streaming the predictor while the ring is full and h is not yet
-// known.  Neurons are dealt round robin to the CTAs (neuron i to CTA i mod G),
+// and issues their gather rows; it keeps issuing P2 tiles meanwhile.  No L2
+// prefetch runs ahead of the ring: prefetched predictor rows queued ahead of
+// the latency-critical P1 and tile loads and made the step slower.
+// Neurons are dealt round robin to the CTAs (neuron i to CTA i mod G),
 // so every CTA gets the same mix of hot and cold neurons; CTA c's k-th tile
 // holds its own neurons c + (32k + q) G, q < 32.  In dense hot-prefix mode the
 // rows of a tile's prefix neurons are issued right after the tile, without
@@ -501,7 +501,7 @@ PI_DEV void producer(Smem &S, const Args &a, int c, int G, int lane) {
     return true;
   };
 
-  // 1. this CTA's rows of P1, then an L2 prefetch of all its P2 rows
+  // 1. this CTA's rows of P1
   for (int j = j0; ok && j < j1; j += rpi) {
     const int n = min(rpi, j1 - j);
     int s;

@@ -217,14 +217,33 @@ def step_bytes(cfg: inputs.Config, B: int, n_union: int) -> int:
 FUSED_SOURCES = ("pi_fused.cuh", "pi_device.cuh")
 
 
+def code_tokens(src: str) -> str:
+    """C/CUDA source with its comments removed and its whitespace collapsed
+    (string and character literals kept as they are): edits to comments or
+    layout leave it unchanged, any edit to the code does not."""
+    import re
+    tok = re.compile(r'"(?:\\.|[^"\\\n])*"|\'(?:\\.|[^\'\\\n])*\'|//[^\n]*|/\*.*?\*/|\s+|[^"\'/\s]+|/', re.S)
+    out = []
+    for m in tok.finditer(src):
+        t = m.group(0)
+        if t.startswith("//") or t.startswith("/*") or t.isspace():
+            if out and out[-1] != " ":
+                out.append(" ")
+        else:
+            out.append(t)
+    return "".join(out).strip()
+
+
 def kernel_source_hash(files=FUSED_SOURCES) -> str:
-    """Hash of the CUDA sources a kernel is built from; a profile summary's
-    counters apply only to the kernel built from the sources it records."""
+    """Hash of the code (comments and layout excluded) of the CUDA sources a
+    kernel is built from; a profile summary's counters apply only to the
+    kernel built from the code it records."""
     import hashlib
     h = hashlib.sha256()
     for name in files:
-        with open(os.path.join(ROOT, "activation_sparse_decode_gemv_b200", "csrc", name), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "activation_sparse_decode_gemv_b200", "csrc", name), encoding="utf-8") as fh:
+            h.update(code_tokens(fh.read()).encode())
+            h.update(b"\0")
     return h.hexdigest()[:16]
 
 

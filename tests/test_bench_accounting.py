@@ -117,3 +117,12 @@ def test_cli_overrides():
     assert bench.parse(["--hot-mode", "index"]).flags == pb.PI_FFN_HOT_INDEX
     cfg = bench.config_of(a)
     assert cfg.bias_norm == "w1" and dataclasses.replace(cfg, bias_norm="pred") == C["opt_tiny_f32"]
+
+
+def test_code_tokens_ignore_comments_only():
+    a = 'int f(int x) {  // sum\n  return x + 1; /* one */ }\nconst char *s = "//";'
+    b = 'int f(int x) {\n  // the successor\n  return x + 1;\n}\nconst char *s = "//";'
+    assert bench.code_tokens(a) == bench.code_tokens(b)
+    # a changed literal or operand is a code change
+    assert bench.code_tokens(a) != bench.code_tokens(a.replace("x + 1", "x + 2"))
+    assert bench.code_tokens(a) != bench.code_tokens(a.replace('"//"', '"/"'))
