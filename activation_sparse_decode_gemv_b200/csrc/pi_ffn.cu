@@ -39,7 +39,8 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Workspace layout for a call at batch B on layers with the given maxima.
 // [0, 256): status region: int status, int union count, grid-barrier word,
-// and (at byte 64) the epoch of the fused kernel's tagged words.
+// at byte 64 the epoch of the fused kernel's tagged words, at byte 68 its
+// arrival counter of the reduction slices.
 // [256, 1024): the batch kernel's per-tile arrival counters (zero between
 // calls; the kernel restores them), at a place that does not move with B.
 // fx_h / fx_part: the fused kernel's tagged exchange words (h, partials of y);
@@ -49,6 +50,7 @@ struct WsLayout {
   int G, a_stride;
 };
 constexpr size_t kEpochOffset = 64;
+constexpr size_t kTicketOffset = 68;
 constexpr size_t kBatchCtrOffset = 256;
 constexpr size_t kHeaderBytes = 1024;
 static_assert(kBatchCtrOffset + pi::batch::kMaxTiles * 4 <= kHeaderBytes, "batch counters fit the header");
@@ -244,6 +246,7 @@ struct Ws {
   int32_t *ulist() const { return reinterpret_cast<int32_t *>(base + L.ulist); }
   float *partial() const { return reinterpret_cast<float *>(base + L.partial); }
   unsigned *epoch() const { return reinterpret_cast<unsigned *>(base + kEpochOffset); }
+  unsigned *ticket() const { return reinterpret_cast<unsigned *>(base + kTicketOffset); }
   unsigned long long *fx_h() const { return reinterpret_cast<unsigned long long *>(base + L.fx_h); }
   unsigned long long *fx_part() const { return reinterpret_cast<unsigned long long *>(base + L.fx_part); }
   __half *b_ahi() const { return reinterpret_cast<__half *>(base + L.b_ahi); }
@@ -851,6 +854,7 @@ pi_status run_fused(const pi_ffn *h, const void *in, float *out, int stack, int 
   a.hx = w.fx_h();
   a.px = w.fx_part();
   a.epoch = w.epoch();
+  a.ticket = w.ticket();
   a.mask32 = w.mask();
   a.bar = w.grid_bar();
   a.status = w.status();

@@ -36,12 +36,13 @@
 // 64-bit word (value bits, tag), stored and loaded with single-copy-atomic
 // relaxed gpu-scope accesses.  The tag is the launch's epoch + 1; the epoch
 // lives in the workspace, every CTA reads it after griddepcontrol.wait, and
-// CTA 0 advances it once its reduction has seen every CTA's partial (so every
-// CTA has read it).  A reader polls until the tag matches, so publishing h or
-// a partial of y costs one L2 round trip and no grid barrier.  After the
-// stream every CTA publishes its fp32 partial of y; each CTA then sums a
-// column slice over all partials in CTA order (deterministic, no atomics) and
-// writes y (or adds it to the residual x).
+// the rank-0 reducer advances it once its reduction has seen every CTA's
+// partial (so every CTA has read it).  A reader polls until the tag matches,
+// so publishing h or a partial of y costs one L2 round trip and no grid
+// barrier.  After the stream every CTA publishes its fp32 partial of y; the
+// CTAs that end their stream first (arrival ticket) each sum a column slice
+// over all partials in CTA order (deterministic, no atomics on y) and write
+// y (or add it to the residual x).
 // Every wait is bounded (about 2 s); on expiry the kernel records
 // PI_ERR_TIMEOUT in the workspace status word and completes.
 #pragma once
@@ -99,6 +100,7 @@ struct Smem {
   double dred[kConsumerWarps];
   float fin[kConsumers / (kRedCols / 2)][kRedCols + 1];
   int iscan[kConsumerWarps];
+  int slice;  // this CTA's reduction slice (its arrival rank at the stream end)
   volatile int abort_flag;
 };
 
@@ -129,6 +131,7 @@ struct Args {
   unsigned long long *hx;  // workspace [r] tagged h
   unsigned long long *px;  // workspace [G x d] tagged partials of y
   unsigned *epoch;         // workspace launch counter of the tags
+  unsigned *ticket;        // workspace arrival counter of the reduction slices
   unsigned *mask32;  // workspace [ceil(f/32)] fired bits of neurons 32w..32w+31, when idx or count != nullptr
   unsigned *bar;     // workspace grid-barrier word (id lists only)
   int *status;
@@ -1068,6 +1071,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
     release(s);
   }
 
+  // arrival ticket, in flight while the partial goes out: the CTAs that end
+  // their stream first sum the slices of y, so a heavily loaded CTA does not
+  // also hold one back (whichever CTA sums a slice adds the partials in CTA
+  // order, so y does not depend on the arrival order)
+  constexpr int kTicketThread = kConsumers - 1;  // fewest column chunks
+  unsigned ticket_raw = 0u;
+  if (tid == kTicketThread) ticket_raw = atomicAdd(a.ticket, 1u);
   if (S.abort_flag && tid == 0) {
     // a wait gave up: let any bulk copy still in flight into this CTA's
     // shared memory land before the CTA can exit (bounded, about 1 ms)
@@ -1090,20 +1100,30 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
     }
   }
 
-  // ---- reduction.  The first R CTAs (R = ceil(d / kRedCols)) each sum a
-  // slice of kRedCols columns over all G partials; the others leave now, so
-  // the next launch's CTAs can take their SMs and start streaming weights
-  // while the reduction runs (the id lists, when asked for, need every CTA).
+  // ---- reduction.  The CTAs with the first R arrival ranks (R =
+  // ceil(d / kRedCols)) each sum the slice of kRedCols columns of their rank
+  // over all G partials; the others leave now, so the next launch's CTAs can
+  // take their SMs and start streaming weights while the reduction runs (the
+  // id lists, when asked for, need every CTA).  The rank is the ticket mod
+  // G, a permutation of 0..G-1 within a launch whatever the counter held;
+  // the holder of rank G - 1 takes G back off, so the counter stays below 2G.
   // Thread (grp, p) = (tid / 32, tid % 32) takes the column pair 2p of the
-  // slice from CTAs grp, grp + 8, ... (in that order), then the 8 group sums
-  // are added in group order: a fixed order, so y is deterministic.
+  // slice from CTAs grp, grp + 16, ... (in that order), then the 16 group
+  // sums are added in group order: a fixed order, so y is deterministic.
+  if (tid == kTicketThread) {
+    const unsigned t = ticket_raw % (unsigned)G;
+    if (t == (unsigned)G - 1u) atomicSub(a.ticket, (unsigned)G);
+    S.slice = (int)t;
+  }
+  consumer_sync();
+  const int sl = S.slice;
   const bool want_ids = a.idx != nullptr || a.count != nullptr;
   const int n_red = (d + kRedCols - 1) / kRedCols;
-  if (c >= n_red && !want_ids) return;
-  if (c < n_red) {
+  if (sl >= n_red && !want_ids) return;
+  if (sl < n_red) {
     constexpr int kGroups = kConsumers / (kRedCols / 2);
     const int pr = tid % (kRedCols / 2), grp = tid / (kRedCols / 2);
-    const int col = c * kRedCols + 2 * pr;
+    const int col = sl * kRedCols + 2 * pr;
     float s0 = 0.f, s1 = 0.f;
     bool timed_out = false;
     if (col < d) {
@@ -1151,17 +1171,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
     S.fin[grp][2 * pr] = s0;
     S.fin[grp][2 * pr + 1] = s1;
     consumer_sync();
-    if (tid < kRedCols && c * kRedCols + tid < d) {
+    if (tid < kRedCols && sl * kRedCols + tid < d) {
       float t = S.fin[0][tid];
 #pragma unroll
       for (int g = 1; g < kGroups; ++g) t += S.fin[g][tid];
-      const int oc = c * kRedCols + tid;
+      const int oc = sl * kRedCols + tid;
       a.out[oc] = (a.stack || a.accumulate) ? a.out[oc] + t : t;
     }
   }
   // every CTA has read the epoch (its partial carries this launch's tag):
-  // advance it for the next launch on this workspace
-  if (c == 0 && tid == 0) st_relaxed_u32(a.epoch, tag);
+  // the rank-0 reducer advances it for the next launch on this workspace
+  if (sl == 0 && tid == 0) st_relaxed_u32(a.epoch, tag);
 
   // ---- ascending active ids (optional): after a grid barrier, CTA c writes
   // the ids of words [c * tpc, (c + 1) * tpc) after the popcount of all

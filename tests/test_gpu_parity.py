@@ -218,6 +218,30 @@ def test_repeated_decode_is_bitwise_stable(cuda_device, name, B):
     assert g.status() == 0
 
 
+@pytest.mark.parametrize("start", [0, 1000003])
+def test_reduction_slices_whatever_the_arrival_counter_holds(cuda_device, start):
+    """Batch 1: the CTAs that finish their stream first sum the slices of y,
+    by their arrival ticket mod the grid size.  From any counter value that
+    is a permutation of the slices, so y is bitwise the same; the counter
+    is back at its start value after every launch."""
+    cfg = inputs.CONFIGS["opt7b_f16"]
+    lt = inputs.make_layer(cfg, layer=cfg.n_layers - 1, seed=0, device="cuda")
+    g = Gpu(lt, 1)
+    u = inputs.layer_input(cfg, inputs.make_tokens(cfg, 0, 1, seed=0).cuda()).cuda()
+    y0 = g.decode(u)[0].clone()  # with the id lists: every CTA stays to the end
+    ticket = g.ws[68:72].view(torch.int32)  # the arrival counter's word in the workspace header
+    assert int(ticket.item()) == 0
+    ticket.fill_(start)
+    y = torch.empty(1, lt.d, device="cuda")
+    for k in range(50):  # without id lists: the CTAs past the last slice leave early
+        y.fill_(float("nan"))
+        pb.pi_decode_ffn(g.layer, u, y, g.ws)
+        assert torch.equal(y, y0), f"launch {k} differs"
+    torch.cuda.synchronize()
+    assert int(ticket.item()) == start
+    assert g.status() == 0
+
+
 # ------------------------------------------------------------------ every batch size of each path
 
 @pytest.mark.parametrize("name,batches", [
