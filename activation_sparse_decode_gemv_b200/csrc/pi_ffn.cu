@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -54,6 +55,28 @@ constexpr size_t kTicketOffset = 68;
 constexpr size_t kBatchCtrOffset = 256;
 constexpr size_t kHeaderBytes = 1024;
 static_assert(kBatchCtrOffset + pi::batch::kMaxTiles * 4 <= kHeaderBytes, "batch counters fit the header");
+
+// A once-per-device setup step (a kernel's function attribute acts on the
+// current device only): one bit per device ordinal below 64.
+class DeviceOnce {
+ public:
+  // runs set() unless it already succeeded on the current device
+  template <typename Set>
+  cudaError_t ensure(Set set) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    const unsigned long long bit = 1ull << dev;
+    if (bits_.load(std::memory_order_acquire) & bit) return cudaSuccess;
+    if ((e = set()) != cudaSuccess) return e;
+    bits_.fetch_or(bit, std::memory_order_acq_rel);
+    return cudaSuccess;
+  }
+
+ private:
+  std::atomic<unsigned long long> bits_{0};
+};
 
 int device_sm_count() {
   int dev = 0, n = 0;
@@ -517,14 +540,13 @@ bool batch_ok(const pi_ffn *h, int B, int G) {
 
 template <int ACT>
 cudaError_t batch_launch(const BK::Args &a, int G, int d, cudaStream_t st) {
-  static int attr_smem = 0;
+  static DeviceOnce attr;
   const int smem = (int)BK::smem_bytes(d, ACT == pi::ACT_SWIGLU ? 2 : 1);
-  if (smem > attr_smem) {
-    cudaError_t e = cudaFuncSetAttribute(BK::ffn_batch_kernel<ACT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         200 * 1024);
-    if (e != cudaSuccess) return e;
-    attr_smem = 200 * 1024;
-  }
+  // the largest size any layer may take (batch_ok), set once per device
+  cudaError_t e = attr.ensure([] {
+    return cudaFuncSetAttribute(BK::ffn_batch_kernel<ACT>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+  });
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(G);
   cfg.blockDim = dim3(BK::kThreads);
@@ -633,13 +655,11 @@ bool tc_ok(const pi_ffn *h, int B) {
 }
 
 template <typename KArg>
-cudaError_t launch_smem(void (*kern)(KArg), int G, int threads, int smem, bool *attr_done, cudaStream_t st,
+cudaError_t launch_smem(void (*kern)(KArg), int G, int threads, int smem, DeviceOnce *attr, cudaStream_t st,
                         const KArg &arg) {
-  if (!*attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    *attr_done = true;
-  }
+  cudaError_t e =
+      attr->ensure([&] { return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem); });
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(G);
   cfg.blockDim = dim3(threads);
@@ -655,14 +675,14 @@ cudaError_t launch_smem(void (*kern)(KArg), int G, int threads, int smem, bool *
 
 template <int KIND, int WT, int ACT>
 cudaError_t ts_launch(const TC::RowArgs &a, int G, cudaStream_t st) {
-  static bool attr = false;
+  static DeviceOnce attr;
   using Sh = TC::RowShape<KIND, WT, ACT>;
   return launch_smem(TC::row_gemm_kernel<KIND, WT, ACT>, G, Sh::THREADS, Sh::SMEM, &attr, st, a);
 }
 
 template <int WT>
 cudaError_t down_launch(const TC::DownArgs &a, int G, cudaStream_t st) {
-  static bool attr = false;
+  static DeviceOnce attr;
   return launch_smem(TC::ffn_down_kernel<WT>, G, TC::kThreads, TC::DownShape<WT>::SMEM, &attr, st, a);
 }
 
@@ -774,18 +794,18 @@ namespace F = pi::fused;
 
 template <int WT, int ACT, int CPT>
 cudaError_t fused_launch(const F::Args &a, int G, cudaStream_t st) {
-  static bool attr_set = false;
+  static DeviceOnce attr;
   const size_t smem = sizeof(F::Smem);
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(F::decode_fused_kernel<WT, ACT, CPT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
+  cudaError_t e = attr.ensure([&] {
+    cudaError_t r = cudaFuncSetAttribute(F::decode_fused_kernel<WT, ACT, CPT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (r != cudaSuccess) return r;
     int nb = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, F::decode_fused_kernel<WT, ACT, CPT>, F::kThreads, smem);
-    if (e != cudaSuccess) return e;
-    if (nb < 1) return cudaErrorInvalidConfiguration;
-    attr_set = true;
-  }
+    r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, F::decode_fused_kernel<WT, ACT, CPT>, F::kThreads, smem);
+    if (r != cudaSuccess) return r;
+    return nb < 1 ? cudaErrorInvalidConfiguration : cudaSuccess;
+  });
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(G);
   cfg.blockDim = dim3(F::kThreads);
