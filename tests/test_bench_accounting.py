@@ -126,3 +126,13 @@ def test_code_tokens_ignore_comments_only():
     # a changed literal or operand is a code change
     assert bench.code_tokens(a) != bench.code_tokens(a.replace("x + 1", "x + 2"))
     assert bench.code_tokens(a) != bench.code_tokens(a.replace('"//"', '"/"'))
+
+
+def test_fused_profile_matches_the_kernel_code():
+    """The committed DRAM-traffic summary was taken on the fused kernel's
+    current code (comments aside), so the bench line can carry its traffic;
+    a code change without a new capture fails here, not silently in the
+    bench line."""
+    t = bench.profiled_traffic("decode_fused_kernel_opt7b_f16_batch1.md")
+    assert t is not None, "profiles/decode_fused_kernel_opt7b_f16_batch1.md predates the kernel code"
+    assert 1.0 <= t / 69.02e6 <= 1.10  # the summary's own algorithmic bytes for that command
